@@ -1,0 +1,424 @@
+"""Pins for the CPU oracle: each test ties it to something other than itself.
+
+The pages give no worked example values for triangular attention, so the
+oracle is pinned by (a) library routines that compute each step
+(torch.nn.functional.layer_norm, matmul, sigmoid,
+torch.nn.functional.scaled_dot_product_attention with an additive mask),
+composed in the order the block defines, (b) closed forms and special cases,
+and (c) invariants: probability rows that sum to one, permutation
+equivariance, the transpose identity between the two orientations, and
+agreement with an online-softmax evaluation of the same attention.
+
+A plausible mistake in the oracle — a dropped bias, a transposed bias index,
+a wrong scale, a missing mean subtraction, a gate applied wrongly, an
+off-by-one key mask — fails at least one of these.
+"""
+import dataclasses
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from protein_pair_representation_layernorm_b200 import workloads
+from conftest import to_problem
+
+pytestmark = pytest.mark.filterwarnings("ignore")
+
+
+def _small(N=9, seed=11, mask="none", c_z=16, H=2, d=4, dtype="f32", chains=()):
+    inp = workloads.make_inputs(N, dtype, seed, mask, chains=chains, c_z=c_z, H=H, d=d)
+    return inp, to_problem(inp)
+
+
+def _nonzero_biases(p: oracle.Problem, seed=5):
+    rng = np.random.default_rng(seed)
+    p.bg = rng.normal(size=p.Wg.shape[0])
+    p.bo = rng.normal(size=p.Wo.shape[0])
+    p.gamma = 1.0 + 0.3 * rng.normal(size=p.c_z)
+    p.beta = 0.2 * rng.normal(size=p.c_z)
+    return p
+
+
+# --------------------------------------------------------------------------
+# Stage-by-stage against library routines
+
+
+def test_layer_norm_matches_torch():
+    rng = np.random.default_rng(0)
+    z = rng.normal(size=(37, 128)) * 3.0 + 1.5
+    gamma = rng.normal(size=128)
+    beta = rng.normal(size=128)
+    x = oracle.layer_norm(z, gamma, beta, 1e-5)
+    ref = F.layer_norm(torch.from_numpy(z), (128,), torch.from_numpy(gamma),
+                       torch.from_numpy(beta), eps=1e-5).numpy()
+    np.testing.assert_allclose(x, ref, rtol=0, atol=1e-12)
+
+
+def test_pair_features_match_matmul():
+    inp, p = _small(N=6)
+    p = _nonzero_biases(p)
+    q, k, v, g, b = oracle.pair_features(p)
+    z = torch.from_numpy(p.Z.astype(np.float64))
+    x = F.layer_norm(z, (p.c_z,), torch.from_numpy(p.gamma), torch.from_numpy(p.beta), eps=p.eps)
+    T = torch.from_numpy
+    np.testing.assert_allclose(q, (x @ T(p.Wq).T).numpy(), atol=1e-12)
+    np.testing.assert_allclose(k, (x @ T(p.Wk).T).numpy(), atol=1e-12)
+    np.testing.assert_allclose(v, (x @ T(p.Wv).T).numpy(), atol=1e-12)
+    np.testing.assert_allclose(g, torch.sigmoid(x @ T(p.Wg).T + T(p.bg)).numpy(), atol=1e-12)
+    # bias[h, a, b] comes from pair (a, b)
+    np.testing.assert_allclose(b, (x @ T(p.Wb).T).permute(2, 0, 1).numpy(), atol=1e-12)
+
+
+def _sdpa(q, k, v, bias, mask):
+    """torch SDPA per head with an additive float mask (bias, -inf for masked keys)."""
+    qt = torch.from_numpy(q).permute(1, 0, 2)      # (H, Nq, d)
+    kt = torch.from_numpy(k).permute(1, 0, 2)
+    vt = torch.from_numpy(v).permute(1, 0, 2)
+    add = torch.from_numpy(bias).clone()           # (H, Nq, Nk)
+    if mask is not None:
+        add[:, :, torch.from_numpy(mask == 0)] = -math.inf
+    o = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=add)
+    return o.permute(1, 0, 2).numpy()
+
+
+@pytest.mark.parametrize("mask", [None, "some"])
+def test_attend_matches_sdpa(mask):
+    rng = np.random.default_rng(1)
+    Nq, Nk, H, d = 13, 17, 3, 8
+    q, k, v = rng.normal(size=(Nq, H, d)), rng.normal(size=(Nk, H, d)), rng.normal(size=(Nk, H, d))
+    bias = rng.normal(size=(H, Nq, Nk)) * 2
+    m = None
+    if mask:
+        m = np.ones(Nk, np.uint8)
+        m[[0, 5, 16]] = 0
+    o = oracle.attend(q, k, v, bias, m)
+    np.testing.assert_allclose(o, _sdpa(q, k, v, bias, m), atol=1e-12)
+
+
+@pytest.mark.parametrize("block", [1, 7, 64])
+def test_attend_blockwise_agrees(block):
+    rng = np.random.default_rng(2)
+    Nq, Nk, H, d = 11, 48, 2, 8
+    q, k, v = rng.normal(size=(Nq, H, d)), rng.normal(size=(Nk, H, d)), rng.normal(size=(Nk, H, d))
+    bias = rng.normal(size=(H, Nq, Nk)) * 3
+    m = np.ones(Nk, np.uint8)
+    m[:9] = 0  # the whole first block of 7 (and more) masked
+    m[30] = 0
+    full = oracle.attend(q, k, v, bias, m)
+    blk = oracle.attend_blockwise(q, k, v, bias, m, block=block)
+    np.testing.assert_allclose(blk, full, atol=1e-12)
+
+
+def test_probabilities_sum_to_one_masked_exactly_zero():
+    rng = np.random.default_rng(3)
+    Nq, Nk, H, d = 9, 21, 2, 4
+    q, k, v = rng.normal(size=(Nq, H, d)), rng.normal(size=(Nk, H, d)), rng.normal(size=(Nk, H, d))
+    bias = rng.normal(size=(H, Nq, Nk)) * 5
+    m = np.ones(Nk, np.uint8)
+    m[[2, 3, 20]] = 0
+    _, P = oracle.attend(q, k, v, bias, m, want_probs=True)
+    np.testing.assert_allclose(P.sum(-1), 1.0, atol=1e-12)
+    assert np.all(P[:, :, m == 0] == 0.0)
+    assert np.all(P[:, :, m == 1] > 0.0)
+
+
+def _block_by_library(p: oracle.Problem, orientation: int) -> np.ndarray:
+    """The whole block composed from library routines (layer_norm, matmul,
+    sigmoid, scaled_dot_product_attention), for both orientations."""
+    T = torch.from_numpy
+    N, H, d, cz = p.N, p.H, p.d, p.c_z
+    z = T(np.asarray(p.Z, dtype=np.float64))
+    if orientation == 1:
+        # the ending node works on columns: view pair (i, j) as (j, i)
+        z = z.transpose(0, 1).contiguous()
+    x = F.layer_norm(z, (cz,), T(p.gamma), T(p.beta), eps=p.eps)
+    q = (x @ T(p.Wq).T).reshape(N, N, H, d)
+    k = (x @ T(p.Wk).T).reshape(N, N, H, d)
+    v = (x @ T(p.Wv).T).reshape(N, N, H, d)
+    g = torch.sigmoid(x @ T(p.Wg).T + (T(p.bg) if p.bg is not None else 0.0))
+    bias = (x @ T(p.Wb).T).permute(2, 0, 1)  # (H, a, b) of the (possibly transposed) view
+    add = bias.clone()
+    if p.mask is not None:
+        add[:, :, T(p.mask == 0)] = -math.inf
+    out = torch.empty_like(z)
+    for a in range(N):
+        # row a of the view: queries (a, j), keys (a, k), bias[h, j, k]
+        o = F.scaled_dot_product_attention(q[a].permute(1, 0, 2), k[a].permute(1, 0, 2),
+                                           v[a].permute(1, 0, 2), attn_mask=add)
+        o = o.permute(1, 0, 2).reshape(N, H * d)
+        if p.mask is not None and not p.mask.any():
+            o = torch.zeros_like(o)
+        out[a] = z[a] + (g[a] * o) @ T(p.Wo).T + (T(p.bo) if p.bo is not None else 0.0)
+    if orientation == 1:
+        out = out.transpose(0, 1)
+    return out.numpy()
+
+
+@pytest.mark.parametrize("orientation", [0, 1])
+@pytest.mark.parametrize("mask", ["none", "random:0.3", "tail:3"])
+def test_block_matches_library_composition(orientation, mask):
+    inp, p = _small(N=10, seed=7, mask=mask)
+    p = _nonzero_biases(p)
+    got = oracle.tri_attn_full(p, orientation)
+    ref = _block_by_library(p, orientation)
+    np.testing.assert_allclose(got, ref, atol=1e-11)
+
+
+@pytest.mark.parametrize("orientation", [0, 1])
+def test_block_matches_library_composition_full_width(orientation):
+    """Same check with the GPU path's widths: c_z = 128, H = 4, d = 32, bf16 inputs."""
+    inp = workloads.make_inputs(12, "bf16", 3, "random:0.25")
+    p = to_problem(inp)
+    got = oracle.tri_attn_full(p, orientation)
+    p64 = to_problem(inp)
+    p64.Z = inp.Z.to(torch.float64).numpy()
+    ref = _block_by_library(p64, orientation)
+    np.testing.assert_allclose(got, ref, atol=1e-11)
+
+
+# --------------------------------------------------------------------------
+# Invariants
+
+
+def test_transpose_identity():
+    """ending(Z) = T(start(T(Z))), the two loops being written independently."""
+    inp, p = _small(N=11, seed=4, mask="random:0.2")
+    p = _nonzero_biases(p)
+    end = oracle.tri_attn_full(p, 1)
+    pt = dataclasses.replace(p)
+    pt.Z = np.ascontiguousarray(np.asarray(p.Z).transpose(1, 0, 2))
+    start_t = oracle.tri_attn_full(pt, 0)
+    np.testing.assert_allclose(end, start_t.transpose(1, 0, 2), atol=1e-12)
+
+
+@pytest.mark.parametrize("orientation", [0, 1])
+def test_permutation_equivariance(orientation):
+    inp, p = _small(N=10, seed=5, mask="random:0.2")
+    p = _nonzero_biases(p)
+    out = oracle.tri_attn_full(p, orientation)
+    perm = np.random.default_rng(9).permutation(p.N)
+    pp = dataclasses.replace(p)
+    pp.Z = np.ascontiguousarray(np.asarray(p.Z)[perm][:, perm])
+    pp.mask = np.ascontiguousarray(p.mask[perm])
+    outp = oracle.tri_attn_full(pp, orientation)
+    np.testing.assert_allclose(outp, out[perm][:, perm], atol=1e-12)
+
+
+def test_ln_shift_invariance():
+    """A constant added to every channel of every pair changes only the
+    residual term (LayerNorm removes the per-pair mean)."""
+    inp, p = _small(N=8, seed=6)
+    p = _nonzero_biases(p)
+    z = np.asarray(p.Z, dtype=np.float64)
+    p.Z = z
+    out = oracle.tri_attn_full(p, 0)
+    ps = dataclasses.replace(p)
+    ps.Z = z + 0.75
+    outs = oracle.tri_attn_full(ps, 0)
+    np.testing.assert_allclose(outs - ps.Z, out - z, atol=1e-11)
+
+
+def test_ln_scale_invariance_eps_zero():
+    """With eps = 0 LayerNorm is invariant to scaling each pair vector."""
+    inp, p = _small(N=7, seed=8)
+    p.eps = 0.0
+    z = np.asarray(p.Z, dtype=np.float64)
+    p.Z = z
+    out = oracle.tri_attn_full(p, 1)
+    ps = dataclasses.replace(p)
+    ps.Z = z * 3.0
+    outs = oracle.tri_attn_full(ps, 1)
+    np.testing.assert_allclose(outs - ps.Z, out - z, atol=1e-11)
+
+
+# --------------------------------------------------------------------------
+# Closed forms and special cases
+
+
+@pytest.mark.parametrize("orientation", [0, 1])
+def test_zero_query_zero_bias_gives_masked_mean(orientation):
+    """Wq = 0 and Wb = 0 make every logit equal, so o_ij is the mean of v over
+    the unmasked keys of the line (row i for the starting node, column j for
+    the ending node)."""
+    inp, p = _small(N=9, seed=10, mask="random:0.3")
+    p = _nonzero_biases(p)
+    p.Wq = np.zeros_like(p.Wq)
+    p.Wb = np.zeros_like(p.Wb)
+    out = oracle.tri_attn_full(p, orientation)
+    q, k, v, g, b = oracle.pair_features(p)
+    valid = p.mask.astype(bool)
+    z = np.asarray(p.Z, dtype=np.float64)
+    exp = np.empty_like(out)
+    for i in range(p.N):
+        for j in range(p.N):
+            if orientation == 0:
+                mean = v[i, valid].mean(0)   # keys (i, k)
+            else:
+                mean = v[valid, j].mean(0)   # keys (k, j)
+            exp[i, j] = z[i, j] + p.Wo @ (g[i, j] * mean) + p.bo
+    np.testing.assert_allclose(out, exp, atol=1e-12)
+
+
+def test_single_pair():
+    """N = 1: the only key is the query's own pair, so o = v and
+    out = z + Wo (g * v) + bo."""
+    inp, p = _small(N=1, seed=12)
+    p = _nonzero_biases(p)
+    q, k, v, g, b = oracle.pair_features(p)
+    z = np.asarray(p.Z, dtype=np.float64)
+    for orientation in (0, 1):
+        out = oracle.tri_attn_full(p, orientation)
+        np.testing.assert_allclose(out[0, 0], z[0, 0] + p.Wo @ (g[0, 0] * v[0, 0]) + p.bo,
+                                   atol=1e-12)
+
+
+@pytest.mark.parametrize("orientation", [0, 1])
+def test_single_valid_key(orientation):
+    inp, p = _small(N=8, seed=13)
+    p = _nonzero_biases(p)
+    kstar = 5
+    p.mask = np.zeros(p.N, np.uint8)
+    p.mask[kstar] = 1
+    out = oracle.tri_attn_full(p, orientation)
+    q, k, v, g, b = oracle.pair_features(p)
+    z = np.asarray(p.Z, dtype=np.float64)
+    for i in range(p.N):
+        for j in range(p.N):
+            vv = v[i, kstar] if orientation == 0 else v[kstar, j]
+            np.testing.assert_allclose(out[i, j], z[i, j] + p.Wo @ (g[i, j] * vv) + p.bo,
+                                       atol=1e-12)
+
+
+@pytest.mark.parametrize("orientation", [0, 1])
+def test_all_keys_masked_returns_input(orientation):
+    inp, p = _small(N=6, seed=14, mask="all")
+    out = oracle.tri_attn_full(p, orientation)  # bo = 0
+    np.testing.assert_array_equal(out, np.asarray(p.Z, dtype=np.float64))
+
+
+def test_zero_output_projection_returns_input():
+    inp, p = _small(N=6, seed=15)
+    p.Wo = np.zeros_like(p.Wo)
+    for orientation in (0, 1):
+        out = oracle.tri_attn_full(p, orientation)
+        np.testing.assert_array_equal(out, np.asarray(p.Z, dtype=np.float64))
+
+
+def test_gate_closed_form():
+    """Wg = 0: the gate is sigmoid(bg).  bg = 0 gives 1/2, bg = ln 3 gives 3/4,
+    so the attention update scales by exactly 3/2."""
+    inp, p = _small(N=7, seed=16)
+    p.Wg = np.zeros_like(p.Wg)
+    p.bg = np.zeros(p.Wg.shape[0])
+    z = np.asarray(p.Z, dtype=np.float64)
+    u_half = oracle.tri_attn_full(p, 0) - z
+    p.bg = np.full(p.Wg.shape[0], math.log(3.0))
+    u_34 = oracle.tri_attn_full(p, 0) - z
+    np.testing.assert_allclose(u_34, 1.5 * u_half, atol=1e-12)
+
+
+@pytest.mark.parametrize("orientation", [0, 1])
+def test_dominant_bias_selects_key(orientation):
+    """Wq = 0 and a bias that is huge on exactly one key per query: the output
+    is the value of that key.  The key is found from the pair-(a, b) bias
+    returned by pair_features, so a transposed bias index in the block fails."""
+    inp, p = _small(N=8, seed=17)
+    p.Wq = np.zeros_like(p.Wq)
+    b0 = oracle.pair_features(p)[4]
+    # scale Wb so that, in every softmax row of either orientation, the top
+    # logit exceeds the runner-up by at least 60 (one-hot to 1e-26)
+    srt = np.sort(np.concatenate([b0, b0.transpose(0, 2, 1)], axis=1), axis=-1)
+    gap = float((srt[..., -1] - srt[..., -2]).min())
+    p.Wb = p.Wb * (60.0 / gap)
+    q, k, v, g, b = oracle.pair_features(p)
+    out = oracle.tri_attn_full(p, orientation)
+    z = np.asarray(p.Z, dtype=np.float64)
+    H, d = p.H, p.d
+    for i in range(p.N):
+        for j in range(p.N):
+            o = np.empty(H * d)
+            for h in range(H):
+                if orientation == 0:
+                    ks = int(np.argmax(b[h, j, :]))          # bias beta_h(j, k)
+                    o[h * d:(h + 1) * d] = v[i, ks, h * d:(h + 1) * d]
+                else:
+                    ks = int(np.argmax(b[h, :, i]))          # bias beta_h(k, i)
+                    o[h * d:(h + 1) * d] = v[ks, j, h * d:(h + 1) * d]
+            np.testing.assert_allclose(out[i, j], z[i, j] + p.Wo @ (g[i, j] * o), atol=1e-9)
+
+
+def test_hand_worked_two_residues():
+    """N = 2, c_z = 4, H = 1, d = 2, eps = 0, worked by hand.
+
+    Every pair vector is a permutation of (1, 1, -1, -1): mean 0, variance 1,
+    so LayerNorm returns it unchanged.  Weights select channels:
+    q = (x0, x1), k = (x2, x3), v = (x0, x2), bias = x1, gate = sigmoid(0) = 1/2,
+    out = z + (o0/2, o1/2, 0, 0).
+        Z00 = ( 1, 1,-1,-1): q=( 1, 1) k=(-1,-1) v=( 1,-1) b= 1
+        Z01 = ( 1,-1, 1,-1): q=( 1,-1) k=( 1,-1) v=( 1, 1) b=-1
+        Z10 = ( 1,-1,-1, 1): q=( 1,-1) k=(-1, 1) v=( 1,-1) b=-1
+        Z11 = (-1, 1, 1,-1): q=(-1, 1) k=( 1,-1) v=(-1, 1) b= 1
+    Starting node, (i, j) = (0, 0): q=(1,1); keys k00=(-1,-1), k01=(1,-1):
+    dots -2, 0; biases beta(0,0)=1, beta(0,1)=-1; logits -2/sqrt2+1, -1.
+    With two keys the softmax is logistic: p0 = 1/(1+exp(l1-l0)).
+    """
+    Z = np.array([[[1, 1, -1, -1], [1, -1, 1, -1]],
+                  [[1, -1, -1, 1], [-1, 1, 1, -1]]], dtype=np.float64)
+    sel = lambda rows: np.array([[1.0 if c == r else 0.0 for c in range(4)] for r in rows])
+    p = oracle.Problem(Z=Z, gamma=np.ones(4), beta=np.zeros(4), Wq=sel([0, 1]), Wk=sel([2, 3]),
+                       Wv=sel([0, 2]), Wg=np.zeros((2, 4)), Wb=sel([1]),
+                       Wo=np.array([[1.0, 0], [0, 1.0], [0, 0], [0, 0]]), H=1, d=2, eps=0.0)
+    r2 = math.sqrt(2.0)
+    lg = lambda l0, l1: 1.0 / (1.0 + math.exp(l1 - l0))
+    # pair features by hand
+    q = {(0, 0): (1, 1), (0, 1): (1, -1), (1, 0): (1, -1), (1, 1): (-1, 1)}
+    k = {(0, 0): (-1, -1), (0, 1): (1, -1), (1, 0): (-1, 1), (1, 1): (1, -1)}
+    v = {(0, 0): (1, -1), (0, 1): (1, 1), (1, 0): (1, -1), (1, 1): (-1, 1)}
+    b = {(0, 0): 1, (0, 1): -1, (1, 0): -1, (1, 1): 1}
+    dot = lambda a, c: a[0] * c[0] + a[1] * c[1]
+    for orientation in (0, 1):
+        out = oracle.tri_attn_full(p, orientation)
+        for i in range(2):
+            for j in range(2):
+                if orientation == 0:   # keys (i, k), bias beta(j, k)
+                    l0 = dot(q[i, j], k[i, 0]) / r2 + b[j, 0]
+                    l1 = dot(q[i, j], k[i, 1]) / r2 + b[j, 1]
+                    va, vb = v[i, 0], v[i, 1]
+                else:                  # keys (k, j), bias beta(k, i)
+                    l0 = dot(q[i, j], k[0, j]) / r2 + b[0, i]
+                    l1 = dot(q[i, j], k[1, j]) / r2 + b[1, i]
+                    va, vb = v[0, j], v[1, j]
+                p0 = lg(l0, l1)
+                o = [p0 * va[c] + (1 - p0) * vb[c] for c in range(2)]
+                exp = Z[i, j] + np.array([o[0] / 2, o[1] / 2, 0.0, 0.0])
+                np.testing.assert_allclose(out[i, j], exp, atol=1e-14)
+    # the one value written out in the docstring
+    out0 = oracle.tri_attn_full(p, 0)
+    p0 = 1.0 / (1.0 + math.exp(-1.0 - (-2.0 / r2 + 1.0)))
+    assert abs(out0[0, 0, 0] - (1.0 + (p0 * 1 + (1 - p0) * 1) / 2)) < 1e-14
+    assert abs(out0[0, 0, 1] - (1.0 + (p0 * -1 + (1 - p0) * 1) / 2)) < 1e-14
+
+
+def test_sampled_lines_equal_full():
+    inp, p = _small(N=9, seed=18, mask="random:0.2")
+    for orientation in (0, 1):
+        full = oracle.tri_attn_full(p, orientation)
+        lines = [0, 8, 3]
+        part = oracle.tri_attn(p, orientation, lines)
+        for r, ln in enumerate(lines):
+            ref = full[ln] if orientation == 0 else full[:, ln]
+            np.testing.assert_array_equal(part[r], ref)
+
+
+def test_workload_recipe_is_deterministic():
+    a = workloads.make_inputs(20, "bf16", 4, "random:0.05")
+    b = workloads.make_inputs(20, "bf16", 4, "random:0.05")
+    assert torch.equal(a.Z.view(torch.int16), b.Z.view(torch.int16))
+    assert torch.equal(a.Wo.float(), b.Wo.float())
+    c = workloads.make_inputs(12, "bf16", 2, chains=(4, 4, 4))
+    z = c.Z.float()
+    # intra-chain blocks carry the +1 offset
+    assert z[:4, :4].mean() > 0.6 and abs(float(z[:4, 4:8].mean())) < 0.4
