@@ -1,0 +1,157 @@
+/*
+ * tri_attn.h — C ABI of the B200 (sm_100a) triangle attention library.
+ *
+ * One call computes the pair-biased triangle attention block over a protein
+ * pair representation Z of shape [N][N][c_z] (channels last), in either the
+ * starting-node or the ending-node orientation:
+ *
+ *   x      = LayerNorm(z)                      per pair, over c_z channels
+ *   q,k,v  = Wq x, Wk x, Wv x                  H heads of width d
+ *   g      = sigmoid(Wg x + bg)
+ *   beta_h = Wb x                              one logit bias per head
+ *   starting node: o_ij = sum_k softmax_k(q_ij.k_ik/sqrt(d) + beta_h(j,k)) v_ik
+ *   ending node:   o_ij = sum_k softmax_k(q_ij.k_kj/sqrt(d) + beta_h(k,i)) v_kj
+ *   out_ij = z_ij + Wo (g_ij * o_ij) + bo
+ *
+ * Sources.  The pair representation (Ns, Ns, Hz), Hz typically 128, as the
+ * bottleneck of protein structure models: LightNobel article
+ * ("蛋白质结构预测模型的量化优化与硬件加速"), §1.1; LayerNorm ahead of the
+ * linear layers and the residual path: same article §2.2.3 (groups A and B)
+ * and §3.1, which also names triangular attention.  Attention scores are
+ * computed tile by tile with an online softmax and never stored as an N x N
+ * matrix: Design-CP technical summary, §Metodología 1 (2D grid sharding,
+ * ring attention).  Kernel fusion of attention to cut memory traffic:
+ * OpenFold-TRT summary, §2 Metodología.  The pages give no equations for
+ * triangular attention; the formulas above are the standard definition of
+ * the block and are what this library computes.
+ *
+ * Masking: mask[k] == 0 removes residue k as a key (probability exactly 0);
+ * rows and columns of masked residues are still computed.  If every key is
+ * masked the attention output is 0 and out = z + bo.
+ *
+ * Threading and streams: calls are asynchronous on the given stream unless
+ * stated otherwise.  A handle is not thread-safe; use one handle per host
+ * thread.  Results are deterministic (no floating-point atomics).
+ * There is no CPU fallback: without a usable sm_100 device every call that
+ * needs one returns TRI_ATTN_ERR_NO_DEVICE.
+ */
+#ifndef TRI_ATTN_H
+#define TRI_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define TRI_ATTN_OK                 0
+#define TRI_ATTN_ERR_INVALID_ARG   -1  /* NULL/misaligned pointer, N < 1, bad enum */
+#define TRI_ATTN_ERR_UNSUPPORTED   -2  /* shape or dtype the kernels do not cover */
+#define TRI_ATTN_ERR_ALIAS         -3  /* out overlaps Z without being equal to it */
+#define TRI_ATTN_ERR_OOM           -4  /* device or host allocation failed */
+#define TRI_ATTN_ERR_CUDA          -5  /* a CUDA runtime call or launch failed */
+#define TRI_ATTN_ERR_TIMEOUT       -6  /* a kernel's bounded wait expired (device status) */
+#define TRI_ATTN_ERR_NO_DEVICE     -7  /* no sm_100 device is available */
+
+/* ---- flags for tri_attn_forward --------------------------------------- */
+#define TRI_ATTN_FLAG_SYNC          1u  /* synchronise the stream and return the device status */
+#define TRI_ATTN_FLAG_TIME_KERNELS  2u  /* record CUDA events around each kernel (see tri_attn_kernel_times) */
+#define TRI_ATTN_FLAG_DEBUG_STALL   4u  /* fault injection: the attention kernel's producer withholds one
+                                           stage, so its consumers' bounded waits expire and the call
+                                           reports TRI_ATTN_ERR_TIMEOUT; nothing faults or traps */
+
+typedef enum { TRI_ATTN_F32 = 0, TRI_ATTN_BF16 = 1 } tri_attn_dtype;
+typedef enum { TRI_ATTN_STARTING = 0, TRI_ATTN_ENDING = 1 } tri_attn_orientation;
+
+typedef struct tri_attn_handle tri_attn_handle;  /* opaque */
+
+/* Weights of one block.  All pointers are DEVICE memory holding `dtype`
+ * elements, row-major, contiguous.  Shapes (out x in):
+ *   ln_gamma, ln_beta [c_z];  w_q, w_k, w_v, w_g [H*d][c_z];  b_g [H*d] or NULL (= 0);
+ *   w_b [H][c_z];  w_o [c_z][H*d];  b_o [c_z] or NULL (= 0).
+ * The kernels are specialised to c_z = 128, H = 4, d = 32; other shapes give
+ * TRI_ATTN_ERR_UNSUPPORTED. */
+typedef struct {
+  int c_z, n_heads, head_dim;
+  tri_attn_dtype dtype;
+  float ln_eps;                 /* LayerNorm epsilon, e.g. 1e-5 */
+  const void *ln_gamma, *ln_beta;
+  const void *w_q, *w_k, *w_v, *w_g;
+  const void *b_g;
+  const void *w_b;
+  const void *w_o;
+  const void *b_o;
+} tri_attn_params;
+
+/* Create a handle on the current CUDA device.  Copies and repacks the weights
+ * into the handle's own device buffers (synchronously), so the caller may
+ * free its copies on return.  *out is set only on TRI_ATTN_OK. */
+int tri_attn_create(const tri_attn_params *params, tri_attn_handle **out);
+
+/* Run the block once on `stream` (a cudaStream_t; NULL = legacy default).
+ *   Z    [N][N][c_z] device, dtype of the handle, 16-byte aligned.
+ *   mask [N] device uint8 (1 = valid key) or NULL (all valid).
+ *   out  [N][N][c_z] device, same dtype; out == Z (in place) is allowed,
+ *        any other overlap returns TRI_ATTN_ERR_ALIAS.
+ * Argument checks happen before any launch; on error nothing is launched.
+ * The handle grows its workspace on demand (cudaMalloc); see
+ * tri_attn_set_workspace_limit.  Returns TRI_ATTN_OK once the kernels are
+ * enqueued, or, with TRI_ATTN_FLAG_SYNC, after the stream has drained, with
+ * the device status of the call. */
+int tri_attn_forward(tri_attn_handle *h, const void *Z, int N, const uint8_t *mask,
+                     tri_attn_orientation orientation, void *out, void *stream,
+                     unsigned flags);
+
+/* End-to-end call on HOST buffers: copies Z (and mask) to the device, applies
+ * the blocks orientations[0], orientations[1], ... in sequence, each on the
+ * output of the previous one (in place in a device staging buffer owned by
+ * the handle), and copies the final result back to out_host.  Synchronous:
+ * returns after out_host is written.  Z_host and out_host may be the same
+ * buffer; pinned host memory gives full PCIe bandwidth. */
+int tri_attn_forward_host(tri_attn_handle *h, const void *Z_host, int N,
+                          const uint8_t *mask_host, const int *orientations,
+                          int n_orientations, void *out_host, void *stream,
+                          unsigned flags);
+
+/* Synchronise `stream` and return the sticky device status of the handle
+ * (TRI_ATTN_OK or TRI_ATTN_ERR_TIMEOUT), then clear it. */
+int tri_attn_get_status(tri_attn_handle *h, void *stream);
+
+/* Device milliseconds spent in each kernel, summed over every launch made
+ * with TRI_ATTN_FLAG_TIME_KERNELS since the previous call of this function
+ * (which resets the record): ms[0] = pair_ln_proj, ms[1] = tri_attn_fwd,
+ * ms[2] = gate_out; launches[k] (may be NULL) = number of launches timed.
+ * Each launch is bracketed by CUDA events on the stream it runs on.
+ * Synchronises on the events. */
+int tri_attn_kernel_times(tri_attn_handle *h, float ms[3], int launches[3]);
+
+/* Upper bound on the workspace (bytes) the handle may allocate; above it the
+ * rows are processed in chunks.  0 restores the default (48 GiB). */
+int tri_attn_set_workspace_limit(tri_attn_handle *h, size_t bytes);
+
+/* Device workspace in bytes that a forward of size N needs without chunking. */
+size_t tri_attn_workspace_bytes(tri_attn_dtype dtype, int N);
+
+/* Device pointers of the intermediate tensors of the last forward call (for
+ * inspection by tests).  Layouts, for rows r of the last chunk and head h:
+ *   q, k, v, o: [rows][H][N][d];  g: [rows][N][H*d];  bias: [H][N][ld_bias]
+ * (bias already scaled by log2(e), -inf at masked keys and at columns >= N;
+ * q already scaled by log2(e)/sqrt(d)).  Element type: bf16 for a BF16
+ * handle, fp32 for F32.  Any output pointer may be NULL. */
+int tri_attn_debug_workspace(tri_attn_handle *h, void **q, void **k, void **v, void **g,
+                             void **bias, void **o, int *ld_bias, int *rows);
+
+/* Release everything the handle owns.  NULL-safe.  Not stream-ordered:
+ * call it after the work that uses the handle has completed. */
+int tri_attn_destroy(tri_attn_handle *h);
+
+/* Static string for a status code. */
+const char *tri_attn_status_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRI_ATTN_H */

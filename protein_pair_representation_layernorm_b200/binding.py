@@ -1,0 +1,259 @@
+"""Thin ctypes binding of the C ABI in include/tri_attn.h.
+
+Each ``tri_attn_*`` function here marshals its arguments and calls the C
+function of the same name; every step of the computation runs in the CUDA
+kernels of ``_lib/libtriattn.so``.  PyTorch is used only to hold device
+memory and to name streams.  There is no CPU fallback: if the library is
+missing or no sm_100 device is present the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+from . import build as _build
+
+TRI_ATTN_OK = 0
+TRI_ATTN_ERR_INVALID_ARG = -1
+TRI_ATTN_ERR_UNSUPPORTED = -2
+TRI_ATTN_ERR_ALIAS = -3
+TRI_ATTN_ERR_OOM = -4
+TRI_ATTN_ERR_CUDA = -5
+TRI_ATTN_ERR_TIMEOUT = -6
+TRI_ATTN_ERR_NO_DEVICE = -7
+
+TRI_ATTN_FLAG_SYNC = 1
+TRI_ATTN_FLAG_TIME_KERNELS = 2
+TRI_ATTN_FLAG_DEBUG_STALL = 4
+
+TRI_ATTN_F32 = 0
+TRI_ATTN_BF16 = 1
+TRI_ATTN_STARTING = 0
+TRI_ATTN_ENDING = 1
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "tri_attn.h")
+
+
+class TriAttnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {tri_attn_status_string(code)} ({code})")
+        self.code = code
+
+
+class tri_attn_params(ctypes.Structure):
+    _fields_ = [
+        ("c_z", ctypes.c_int), ("n_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+        ("dtype", ctypes.c_int),
+        ("ln_eps", ctypes.c_float),
+        ("ln_gamma", ctypes.c_void_p), ("ln_beta", ctypes.c_void_p),
+        ("w_q", ctypes.c_void_p), ("w_k", ctypes.c_void_p), ("w_v", ctypes.c_void_p),
+        ("w_g", ctypes.c_void_p),
+        ("b_g", ctypes.c_void_p),
+        ("w_b", ctypes.c_void_p),
+        ("w_o", ctypes.c_void_p),
+        ("b_o", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def lib() -> ctypes.CDLL:
+    """Load (building first if the sources are newer) the CUDA library."""
+    global _lib
+    if _lib is None:
+        path = _build.build() if _build.needs_build() else _build.LIB
+        if not os.path.exists(path):
+            raise RuntimeError(f"CUDA extension missing: {path}")
+        L = ctypes.CDLL(path)
+        vp, ci, cu, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t
+        L.tri_attn_create.argtypes = [ctypes.POINTER(tri_attn_params), ctypes.POINTER(vp)]
+        L.tri_attn_forward.argtypes = [vp, vp, ci, vp, ci, vp, vp, cu]
+        L.tri_attn_forward_host.argtypes = [vp, vp, ci, vp, vp, ci, vp, vp, cu]
+        L.tri_attn_get_status.argtypes = [vp, vp]
+        L.tri_attn_kernel_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float),
+                                            ctypes.POINTER(ctypes.c_int)]
+        L.tri_attn_set_workspace_limit.argtypes = [vp, sz]
+        L.tri_attn_workspace_bytes.argtypes = [ci, ci]
+        L.tri_attn_workspace_bytes.restype = sz
+        L.tri_attn_debug_workspace.argtypes = [vp] + [ctypes.POINTER(vp)] * 6 + [
+            ctypes.POINTER(ci), ctypes.POINTER(ci)]
+        L.tri_attn_destroy.argtypes = [vp]
+        L.tri_attn_status_string.argtypes = [ci]
+        L.tri_attn_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def declared_functions() -> list[str]:
+    """Names of the functions include/tri_attn.h declares."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(tri_attn_[a-z_]+)\s*\(", text)))
+
+
+# ---------------------------------------------------------------- C ABI calls
+
+def tri_attn_status_string(code: int) -> str:
+    return lib().tri_attn_status_string(int(code)).decode()
+
+
+def tri_attn_workspace_bytes(dtype: int, N: int) -> int:
+    return int(lib().tri_attn_workspace_bytes(int(dtype), int(N)))
+
+
+def tri_attn_create(params: tri_attn_params) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    rc = lib().tri_attn_create(ctypes.byref(params), ctypes.byref(h))
+    if rc != TRI_ATTN_OK:
+        raise TriAttnError(rc, "tri_attn_create")
+    return h
+
+
+def tri_attn_forward(h, Z_ptr: int, N: int, mask_ptr, orientation: int, out_ptr: int,
+                     stream: int = 0, flags: int = 0) -> int:
+    return lib().tri_attn_forward(h, Z_ptr, int(N), mask_ptr, int(orientation), out_ptr, stream,
+                                  int(flags))
+
+
+def tri_attn_forward_host(h, Z_host_ptr: int, N: int, mask_host_ptr, orientations,
+                          out_host_ptr: int, stream: int = 0, flags: int = 0) -> int:
+    arr = (ctypes.c_int * len(orientations))(*[int(o) for o in orientations])
+    return lib().tri_attn_forward_host(h, Z_host_ptr, int(N), mask_host_ptr, arr,
+                                       len(orientations), out_host_ptr, stream, int(flags))
+
+
+def tri_attn_get_status(h, stream: int = 0) -> int:
+    return lib().tri_attn_get_status(h, stream)
+
+
+def tri_attn_kernel_times(h) -> tuple[list[float], list[int]]:
+    ms = (ctypes.c_float * 3)()
+    n = (ctypes.c_int * 3)()
+    rc = lib().tri_attn_kernel_times(h, ms, n)
+    if rc != TRI_ATTN_OK:
+        raise TriAttnError(rc, "tri_attn_kernel_times")
+    return [float(x) for x in ms], [int(x) for x in n]
+
+
+def tri_attn_set_workspace_limit(h, nbytes: int) -> int:
+    return lib().tri_attn_set_workspace_limit(h, int(nbytes))
+
+
+def tri_attn_debug_workspace(h) -> dict:
+    ptrs = [ctypes.c_void_p() for _ in range(6)]
+    ld, rows = ctypes.c_int(), ctypes.c_int()
+    rc = lib().tri_attn_debug_workspace(h, *[ctypes.byref(p) for p in ptrs], ctypes.byref(ld),
+                                        ctypes.byref(rows))
+    if rc != TRI_ATTN_OK:
+        raise TriAttnError(rc, "tri_attn_debug_workspace")
+    names = ["q", "k", "v", "g", "bias", "o"]
+    d = {n: p.value for n, p in zip(names, ptrs)}
+    d["ld_bias"] = ld.value
+    d["rows"] = rows.value
+    return d
+
+
+def tri_attn_destroy(h) -> int:
+    return lib().tri_attn_destroy(h)
+
+
+# ---------------------------------------------------------------- convenience
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+class TriangleAttention:
+    """One block's weights on the device plus its handle.
+
+    ``weights`` maps gamma, beta, Wq, Wk, Wv, Wg, bg, Wb, Wo, bo to tensors
+    (any device; they are copied to the current CUDA device in ``dtype``)."""
+
+    def __init__(self, weights: dict, dtype: torch.dtype = torch.bfloat16, eps: float = 1e-5):
+        if dtype not in (torch.float32, torch.bfloat16):
+            raise ValueError("dtype must be float32 or bfloat16")
+        self.dtype = dtype
+        dev = torch.device("cuda", torch.cuda.current_device())
+        self._w = {k: v.detach().to(dev, dtype).contiguous() for k, v in weights.items()
+                   if v is not None}
+        w = self._w
+        p = tri_attn_params()
+        p.c_z, p.n_heads = w["Wo"].shape[0], w["Wb"].shape[0]
+        p.head_dim = w["Wq"].shape[0] // p.n_heads
+        p.dtype = TRI_ATTN_F32 if dtype == torch.float32 else TRI_ATTN_BF16
+        p.ln_eps = eps
+        p.ln_gamma, p.ln_beta = w["gamma"].data_ptr(), w["beta"].data_ptr()
+        p.w_q, p.w_k, p.w_v, p.w_g = (w[k].data_ptr() for k in ("Wq", "Wk", "Wv", "Wg"))
+        p.b_g = w["bg"].data_ptr() if "bg" in w else None
+        p.w_b, p.w_o = w["Wb"].data_ptr(), w["Wo"].data_ptr()
+        p.b_o = w["bo"].data_ptr() if "bo" in w else None
+        self.handle = tri_attn_create(p)
+
+    def forward(self, Z: torch.Tensor, orientation: int = TRI_ATTN_STARTING, mask=None,
+                out: torch.Tensor | None = None, stream=None, flags: int = 0) -> torch.Tensor:
+        assert Z.is_cuda and Z.dtype == self.dtype and Z.is_contiguous()
+        N = Z.shape[0]
+        if out is None:
+            out = torch.empty_like(Z)
+        if mask is not None:
+            mask = mask.to(device=Z.device, dtype=torch.uint8).contiguous()
+        rc = tri_attn_forward(self.handle, _ptr(Z), N, _ptr(mask), orientation, _ptr(out),
+                              _stream_handle(stream), flags)
+        if rc != TRI_ATTN_OK:
+            raise TriAttnError(rc, "tri_attn_forward")
+        return out
+
+    __call__ = forward
+
+    def forward_host(self, Z_host: torch.Tensor, orientations, mask=None,
+                     out: torch.Tensor | None = None, stream=None, flags: int = 0):
+        assert not Z_host.is_cuda and Z_host.is_contiguous()
+        if out is None:
+            out = torch.empty_like(Z_host)
+        if mask is not None:
+            mask = mask.to(torch.uint8).contiguous()
+        rc = tri_attn_forward_host(self.handle, _ptr(Z_host), Z_host.shape[0], _ptr(mask),
+                                   list(orientations), _ptr(out), _stream_handle(stream), flags)
+        if rc != TRI_ATTN_OK:
+            raise TriAttnError(rc, "tri_attn_forward_host")
+        return out
+
+    def status(self, stream=None) -> int:
+        return tri_attn_get_status(self.handle, _stream_handle(stream))
+
+    def kernel_times(self) -> tuple[list[float], list[int]]:
+        """(ms per kernel, launches per kernel) since the previous call."""
+        return tri_attn_kernel_times(self.handle)
+
+    def set_workspace_limit(self, nbytes: int):
+        rc = tri_attn_set_workspace_limit(self.handle, nbytes)
+        if rc != TRI_ATTN_OK:
+            raise TriAttnError(rc, "tri_attn_set_workspace_limit")
+
+    def debug_workspace(self) -> dict:
+        return tri_attn_debug_workspace(self.handle)
+
+    def close(self):
+        if getattr(self, "handle", None) is not None:
+            tri_attn_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

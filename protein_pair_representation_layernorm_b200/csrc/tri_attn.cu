@@ -1,0 +1,736 @@
+// tri_attn.cu — host side of the C ABI declared in include/tri_attn.h, and the
+// single translation unit that instantiates every kernel of the library.
+//
+// A forward call is three kernels on the caller's stream:
+//   pair_ln_proj  (LayerNorm + Q/K/V/gate/bias, tcgen05)        HBM-bound
+//   tri_attn_fwd  (online-softmax attention, tcgen05 + TMA)     tensor/ALU-bound
+//   gate_out      (gate * o, output projection, residual)       HBM-bound
+// (fp32 handles run the SIMT kernels of kernels_f32.cuh instead).  The logit
+// bias of every pair is needed by every row, so it is produced for all pairs
+// before any attention runs; when the workspace for all rows exceeds the
+// handle's limit, a bias-only pass runs first and the rest proceeds in row
+// chunks.
+#include "../../include/tri_attn.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+#include "gate_out.cuh"
+#include "kernels_f32.cuh"
+#include "pair_ln_proj.cuh"
+#include "sm100.cuh"
+#include "tri_attn_fwd.cuh"
+
+namespace {
+
+using bf16 = __nv_bfloat16;
+using tri::kCz;
+using tri::kD;
+using tri::kHD;
+using tri::kHeads;
+
+constexpr size_t kDefaultWorkspaceLimit = size_t(48) << 30;
+
+bool log_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("TRIATTN_LOG");
+    v = (e && e[0] && e[0] != '0') ? 1 : 0;
+  }
+  return v == 1;
+}
+
+#define TA_LOG(...)                                   \
+  do {                                                \
+    if (log_enabled()) {                              \
+      std::fprintf(stderr, "[triattn] " __VA_ARGS__); \
+      std::fprintf(stderr, "\n");                     \
+    }                                                 \
+  } while (0)
+
+#define CUDA_TRY(expr)                                                     \
+  do {                                                                     \
+    cudaError_t err__ = (expr);                                            \
+    if (err__ != cudaSuccess) {                                            \
+      TA_LOG("%s failed: %s", #expr, cudaGetErrorString(err__));           \
+      return err__ == cudaErrorMemoryAllocation ? TRI_ATTN_ERR_OOM          \
+                                                : TRI_ATTN_ERR_CUDA;        \
+    }                                                                      \
+  } while (0)
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 tensor map; dims/strides innermost first, strides in bytes (dims 1, 2).
+bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                 uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {s1, s2};
+  const cuuint32_t box[3] = {b0, b1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) TA_LOG("cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ weight packing
+uint16_t f32_to_bf16_bits(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  if ((u & 0x7fffffffu) > 0x7f800000u) return static_cast<uint16_t>((u >> 16) | 0x40);  // NaN
+  u += 0x7fffu + ((u >> 16) & 1u);  // round to nearest even
+  return static_cast<uint16_t>(u >> 16);
+}
+
+float bf16_bits_to_f32(uint16_t b) {
+  uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+// Shared-memory image of a K-major bf16 MMA operand with 128-byte swizzle:
+// rows n of 128 K-elements, split into two 64-element K slabs of rows x 128 B;
+// the 16-byte chunk c of row n sits at chunk position c ^ (n % 8).
+void pack_kmajor_sw128(const std::vector<uint16_t>& w, int rows, std::vector<uint16_t>& img) {
+  img.assign(static_cast<size_t>(rows) * 128, 0);
+  for (int n = 0; n < rows; ++n)
+    for (int k = 0; k < 128; ++k) {
+      const int slab = k / 64, c = (k % 64) / 8, e = k % 8;
+      const size_t byte = static_cast<size_t>(slab) * rows * 128 + static_cast<size_t>(n) * 128 +
+                          ((c ^ (n & 7)) * 16) + e * 2;
+      img[byte / 2] = w[static_cast<size_t>(n) * 128 + k];
+    }
+}
+
+int copy_to_host_f32(const void* dev, size_t n, tri_attn_dtype dt, std::vector<float>& out,
+                     float fill) {
+  out.assign(n, fill);
+  if (!dev) return TRI_ATTN_OK;
+  if (dt == TRI_ATTN_F32) {
+    CUDA_TRY(cudaMemcpy(out.data(), dev, n * 4, cudaMemcpyDeviceToHost));
+  } else {
+    std::vector<uint16_t> tmp(n);
+    CUDA_TRY(cudaMemcpy(tmp.data(), dev, n * 2, cudaMemcpyDeviceToHost));
+    for (size_t k = 0; k < n; ++k) out[k] = bf16_bits_to_f32(tmp[k]);
+  }
+  return TRI_ATTN_OK;
+}
+
+template <class T>
+int upload(const std::vector<T>& v, void** dst) {
+  CUDA_TRY(cudaMalloc(dst, v.size() * sizeof(T)));
+  CUDA_TRY(cudaMemcpy(*dst, v.data(), v.size() * sizeof(T), cudaMemcpyHostToDevice));
+  return TRI_ATTN_OK;
+}
+
+bool attrs_set = false;
+
+int set_kernel_attrs() {
+  if (attrs_set) return TRI_ATTN_OK;
+  CUDA_TRY(cudaFuncSetAttribute(tri::plp::kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                tri::plp::kSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(tri::attn::kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                tri::attn::kSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(tri::gout::kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                tri::gout::kSmemBytes));
+  attrs_set = true;
+  return TRI_ATTN_OK;
+}
+
+struct EventPair {
+  cudaEvent_t a = nullptr, b = nullptr;
+};
+
+}  // namespace
+
+struct tri_attn_handle {
+  int device = 0;
+  int num_sms = 148;
+  tri_attn_dtype dtype = TRI_ATTN_BF16;
+  float eps = 1e-5f;
+  float q_scale = 0.f;
+  // packed weights (device)
+  void* w_qkvg = nullptr;  // bf16: MMA B image (128 KB); f32: [512][128]
+  void* w_o = nullptr;     // bf16: MMA B image (32 KB);  f32: [128][128]
+  float* w_b = nullptr;    // [H][c_z], times log2(e)
+  float* gamma = nullptr;
+  float* beta = nullptr;
+  float* b_g = nullptr;
+  float* b_o = nullptr;
+  int* status = nullptr;   // device status word
+  // workspace
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  size_t ws_limit = kDefaultWorkspaceLimit;
+  // last forward, for tri_attn_debug_workspace
+  void *q = nullptr, *k = nullptr, *v = nullptr, *g = nullptr, *bias = nullptr, *o = nullptr;
+  int ld_bias = 0, rows_last = 0;
+  // host-buffer entry point staging
+  void* stage = nullptr;
+  size_t stage_bytes = 0;
+  uint8_t* stage_mask = nullptr;
+  size_t stage_mask_bytes = 0;
+  // kernel timing
+  std::vector<EventPair> ev[3];
+  int ev_used[3] = {0, 0, 0};
+};
+
+namespace {
+
+size_t esize(tri_attn_dtype dt) { return dt == TRI_ATTN_F32 ? 4 : 2; }
+
+int ld_bias_for(int N) { return static_cast<int>(align_up(static_cast<size_t>(N), 64)); }
+
+size_t bias_bytes(tri_attn_dtype dt, int N) {
+  return align_up(static_cast<size_t>(kHeads) * N * ld_bias_for(N) * esize(dt), 256);
+}
+
+size_t row_bytes(tri_attn_dtype dt, int N) {
+  // Q, K, V, O: H*d per pair; G: H*d per pair
+  return static_cast<size_t>(N) * 5 * kHD * esize(dt);
+}
+
+struct Layout {
+  size_t q, k, v, g, o, bias, total;
+};
+
+Layout layout_for(tri_attn_dtype dt, int N, int rows) {
+  Layout L{};
+  const size_t per = align_up(static_cast<size_t>(rows) * N * kHD * esize(dt), 256);
+  L.q = 0;
+  L.k = per;
+  L.v = 2 * per;
+  L.g = 3 * per;
+  L.o = 4 * per;
+  L.bias = 5 * per;
+  L.total = L.bias + bias_bytes(dt, N);
+  return L;
+}
+
+int ensure_workspace(tri_attn_handle* h, size_t bytes) {
+  if (h->ws_bytes >= bytes) return TRI_ATTN_OK;
+  if (h->ws) cudaFree(h->ws);
+  h->ws = nullptr;
+  h->ws_bytes = 0;
+  CUDA_TRY(cudaMalloc(&h->ws, bytes));
+  h->ws_bytes = bytes;
+  return TRI_ATTN_OK;
+}
+
+EventPair& timing_slot(tri_attn_handle* h, int kernel) {
+  int& used = h->ev_used[kernel];
+  auto& vec = h->ev[kernel];
+  if (used == static_cast<int>(vec.size())) {
+    EventPair p;
+    cudaEventCreate(&p.a);
+    cudaEventCreate(&p.b);
+    vec.push_back(p);
+  }
+  return vec[used++];
+}
+
+struct Timer {
+  tri_attn_handle* h;
+  cudaStream_t st;
+  bool on;
+  EventPair* p = nullptr;
+  Timer(tri_attn_handle* h_, cudaStream_t s, bool on_, int kernel) : h(h_), st(s), on(on_) {
+    if (on) {
+      p = &timing_slot(h, kernel);
+      cudaEventRecord(p->a, st);
+    }
+  }
+  ~Timer() {
+    if (on) cudaEventRecord(p->b, st);
+  }
+};
+
+bool ranges_overlap(const void* a, const void* b, size_t bytes) {
+  const char* x = static_cast<const char*>(a);
+  const char* y = static_cast<const char*>(b);
+  return x < y + bytes && y < x + bytes;
+}
+
+int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, int orient,
+                 void* out, cudaStream_t st, unsigned flags) {
+  const tri_attn_dtype dt = h->dtype;
+  const bool timed = (flags & TRI_ATTN_FLAG_TIME_KERNELS) != 0;
+  const int ld = ld_bias_for(N);
+
+  // rows per chunk under the workspace limit
+  const size_t full = layout_for(dt, N, N).total;
+  int rows = N;
+  if (full > h->ws_limit) {
+    const size_t fixed = bias_bytes(dt, N) + 6 * 256;
+    if (h->ws_limit <= fixed) return TRI_ATTN_ERR_OOM;
+    size_t fit = (h->ws_limit - fixed) / row_bytes(dt, N);
+    fit = fit / tri::attn::kRows * tri::attn::kRows;
+    if (fit < static_cast<size_t>(tri::attn::kRows)) return TRI_ATTN_ERR_OOM;
+    rows = static_cast<int>(std::min<size_t>(fit, static_cast<size_t>(N)));
+  }
+  const bool chunked = rows < N;
+  const Layout L = layout_for(dt, N, rows);
+  int rc = ensure_workspace(h, L.total);
+  if (rc != TRI_ATTN_OK) return rc;
+  char* ws = static_cast<char*>(h->ws);
+  h->q = ws + L.q;
+  h->k = ws + L.k;
+  h->v = ws + L.v;
+  h->g = ws + L.g;
+  h->o = ws + L.o;
+  h->bias = ws + L.bias;
+  h->ld_bias = ld;
+  TA_LOG("forward N=%d orient=%d dtype=%d rows/chunk=%d ws=%zu", N, orient, static_cast<int>(dt),
+         rows, L.total);
+
+  if (dt == TRI_ATTN_F32) {
+    const float* Zf = static_cast<const float*>(Z);
+    float* outf = static_cast<float*>(out);
+    const int pad = ld - N;
+    if (pad > 0) {
+      const long long tot = static_cast<long long>(kHeads) * N * pad;
+      tri::f32::bias_pad_kernel<<<static_cast<unsigned>((tot + 255) / 256), 256, 0, st>>>(
+          static_cast<float*>(h->bias), N, ld);
+    }
+    auto proj = [&](int row0, int nrows, int wq, int wb) {
+      tri::ProjArgsF32 a{};
+      a.Z = Zf;
+      a.mask = mask;
+      a.N = N;
+      a.orient = orient;
+      a.row0 = row0;
+      a.rows = nrows;
+      a.write_qkvg = wq;
+      a.write_bias = wb;
+      a.w_qkvg = static_cast<const float*>(h->w_qkvg);
+      a.w_b = h->w_b;
+      a.gamma = h->gamma;
+      a.beta = h->beta;
+      a.b_g = h->b_g;
+      a.eps = h->eps;
+      a.q_scale = h->q_scale;
+      a.Q = static_cast<float*>(h->q);
+      a.K = static_cast<float*>(h->k);
+      a.V = static_cast<float*>(h->v);
+      a.G = static_cast<float*>(h->g);
+      a.bias = static_cast<float*>(h->bias);
+      a.ld_bias = ld;
+      const long long pairs = static_cast<long long>(nrows) * N;
+      Timer tm(h, st, timed, 0);
+      tri::f32::ln_proj_kernel<<<static_cast<unsigned>((pairs + tri::f32::kProjThreads - 1) /
+                                                        tri::f32::kProjThreads),
+                                 tri::f32::kProjThreads, 0, st>>>(a);
+    };
+    if (chunked) proj(0, N, 0, 1);
+    for (int r0 = 0; r0 < N; r0 += rows) {
+      const int nr = std::min(rows, N - r0);
+      proj(r0, nr, 1, chunked ? 0 : 1);
+      {
+        tri::AttnArgsF32 a{};
+        a.Q = static_cast<const float*>(h->q);
+        a.K = static_cast<const float*>(h->k);
+        a.V = static_cast<const float*>(h->v);
+        a.bias = static_cast<const float*>(h->bias);
+        a.O = static_cast<float*>(h->o);
+        a.N = N;
+        a.rows = nr;
+        a.ld_bias = ld;
+        const long long tot = static_cast<long long>(nr) * kHeads * N;
+        Timer tm(h, st, timed, 1);
+        tri::f32::attn_kernel<<<static_cast<unsigned>((tot + 127) / 128), 128, 0, st>>>(a);
+      }
+      {
+        tri::GateArgsF32 a{};
+        a.Z = Zf;
+        a.O = static_cast<const float*>(h->o);
+        a.G = static_cast<const float*>(h->g);
+        a.w_o = static_cast<const float*>(h->w_o);
+        a.b_o = h->b_o;
+        a.out = outf;
+        a.N = N;
+        a.orient = orient;
+        a.row0 = r0;
+        a.rows = nr;
+        const long long pairs = static_cast<long long>(nr) * N;
+        Timer tm(h, st, timed, 2);
+        tri::f32::gate_out_kernel<<<static_cast<unsigned>((pairs + tri::f32::kProjThreads - 1) /
+                                                          tri::f32::kProjThreads),
+                                    tri::f32::kProjThreads, 0, st>>>(a);
+      }
+    }
+    h->rows_last = std::min(rows, N - (N - 1) / rows * rows);
+    CUDA_TRY(cudaGetLastError());
+    return TRI_ATTN_OK;
+  }
+
+  // ------------------------------------------------------------ bf16 path
+  rc = set_kernel_attrs();
+  if (rc != TRI_ATTN_OK) return rc;
+  const bf16* Zb = static_cast<const bf16*>(Z);
+  bf16* outb = static_cast<bf16*>(out);
+  const int jtiles = (N + 127) / 128;
+  auto proj = [&](int row0, int nrows, int wq, int wb) {
+    tri::ProjArgs a{};
+    a.Z = Zb;
+    a.mask = mask;
+    a.N = N;
+    a.orient = orient;
+    a.row0 = row0;
+    a.rows = nrows;
+    a.write_qkvg = wq;
+    a.write_bias = wb;
+    a.w_img = static_cast<const uint8_t*>(h->w_qkvg);
+    a.w_b = h->w_b;
+    a.gamma = h->gamma;
+    a.beta = h->beta;
+    a.b_g = h->b_g;
+    a.eps = h->eps;
+    a.q_scale = h->q_scale;
+    a.Q = static_cast<bf16*>(h->q);
+    a.K = static_cast<bf16*>(h->k);
+    a.V = static_cast<bf16*>(h->v);
+    a.G = static_cast<bf16*>(h->g);
+    a.bias = static_cast<bf16*>(h->bias);
+    a.ld_bias = ld;
+    a.status = h->status;
+    const long long ntiles = static_cast<long long>(nrows) * jtiles;
+    const unsigned grid = static_cast<unsigned>(std::min<long long>(ntiles, h->num_sms));
+    Timer tm(h, st, timed, 0);
+    tri::plp::kernel<<<grid, tri::plp::kThreads, tri::plp::kSmemBytes, st>>>(a);
+  };
+  if (chunked) proj(0, N, 0, 1);
+  for (int r0 = 0; r0 < N; r0 += rows) {
+    const int nr = std::min(rows, N - r0);
+    proj(r0, nr, 1, chunked ? 0 : 1);
+    {
+      CUtensorMap mq, mk, mv, mb;
+      const uint64_t rh = static_cast<uint64_t>(nr) * kHeads;
+      const uint64_t row_stride = static_cast<uint64_t>(N) * kD * 2;
+      bool okm = make_map_3d(&mq, h->q, kD, N, rh, kD * 2, row_stride, kD, tri::attn::kBJ,
+                             CU_TENSOR_MAP_SWIZZLE_64B) &&
+                 make_map_3d(&mk, h->k, kD, N, rh, kD * 2, row_stride, kD, tri::attn::kBK,
+                             CU_TENSOR_MAP_SWIZZLE_64B) &&
+                 make_map_3d(&mv, h->v, kD, N, rh, kD * 2, row_stride, kD, tri::attn::kBK,
+                             CU_TENSOR_MAP_SWIZZLE_64B) &&
+                 make_map_3d(&mb, h->bias, ld, N, kHeads, static_cast<uint64_t>(ld) * 2,
+                             static_cast<uint64_t>(N) * ld * 2, tri::attn::kBK, tri::attn::kBJ,
+                             CU_TENSOR_MAP_SWIZZLE_128B);
+      if (!okm) return TRI_ATTN_ERR_CUDA;
+      tri::AttnArgs a{};
+      a.O = static_cast<bf16*>(h->o);
+      a.N = N;
+      a.rows = nr;
+      a.debug_stall = (flags & TRI_ATTN_FLAG_DEBUG_STALL) ? 1 : 0;
+      a.status = h->status;
+      dim3 grid(jtiles, (nr + tri::attn::kRows - 1) / tri::attn::kRows, kHeads);
+      Timer tm(h, st, timed, 1);
+      tri::attn::kernel<<<grid, tri::attn::kThreads, tri::attn::kSmemBytes, st>>>(mq, mk, mv, mb,
+                                                                                 a);
+    }
+    {
+      tri::GateArgs a{};
+      a.Z = Zb;
+      a.O = static_cast<const bf16*>(h->o);
+      a.G = static_cast<const bf16*>(h->g);
+      a.wo_img = static_cast<const uint8_t*>(h->w_o);
+      a.b_o = h->b_o;
+      a.out = outb;
+      a.N = N;
+      a.orient = orient;
+      a.row0 = r0;
+      a.rows = nr;
+      a.status = h->status;
+      dim3 grid(jtiles, nr);
+      Timer tm(h, st, timed, 2);
+      tri::gout::kernel<<<grid, tri::gout::kThreads, tri::gout::kSmemBytes, st>>>(a);
+    }
+  }
+  h->rows_last = N - (N - 1) / rows * rows;
+  CUDA_TRY(cudaGetLastError());
+  return TRI_ATTN_OK;
+}
+
+int read_status(tri_attn_handle* h, cudaStream_t st) {
+  int s = 0;
+  CUDA_TRY(cudaMemcpyAsync(&s, h->status, sizeof(int), cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaStreamSynchronize(st));
+  if (s != 0) CUDA_TRY(cudaMemsetAsync(h->status, 0, sizeof(int), st));
+  CUDA_TRY(cudaStreamSynchronize(st));
+  return s;
+}
+
+int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return TRI_ATTN_ERR_NO_DEVICE;
+  }
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return TRI_ATTN_ERR_NO_DEVICE;
+  }
+  return major == 10 ? TRI_ATTN_OK : TRI_ATTN_ERR_NO_DEVICE;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tri_attn_status_string(int code) {
+  switch (code) {
+    case TRI_ATTN_OK: return "ok";
+    case TRI_ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case TRI_ATTN_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case TRI_ATTN_ERR_ALIAS: return "out partially overlaps Z";
+    case TRI_ATTN_ERR_OOM: return "out of memory";
+    case TRI_ATTN_ERR_CUDA: return "CUDA error";
+    case TRI_ATTN_ERR_TIMEOUT: return "device wait timed out";
+    case TRI_ATTN_ERR_NO_DEVICE: return "no sm_100 device";
+    default: return "unknown status";
+  }
+}
+
+size_t tri_attn_workspace_bytes(tri_attn_dtype dtype, int N) {
+  if (N < 1 || (dtype != TRI_ATTN_F32 && dtype != TRI_ATTN_BF16)) return 0;
+  return layout_for(dtype, N, N).total;
+}
+
+int tri_attn_create(const tri_attn_params* p, tri_attn_handle** out) {
+  if (!p || !out) return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->dtype != TRI_ATTN_F32 && p->dtype != TRI_ATTN_BF16) return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->c_z != kCz || p->n_heads != kHeads || p->head_dim != kD) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (!p->ln_gamma || !p->ln_beta || !p->w_q || !p->w_k || !p->w_v || !p->w_g || !p->w_b ||
+      !p->w_o)
+    return TRI_ATTN_ERR_INVALID_ARG;
+  if (!(p->ln_eps >= 0.f) || !std::isfinite(p->ln_eps)) return TRI_ATTN_ERR_INVALID_ARG;
+  int rc = check_device();
+  if (rc != TRI_ATTN_OK) return rc;
+
+  tri_attn_handle* h = new (std::nothrow) tri_attn_handle();
+  if (!h) return TRI_ATTN_ERR_OOM;
+  auto fail = [&](int code) {
+    tri_attn_destroy(h);
+    return code;
+  };
+  cudaGetDevice(&h->device);
+  cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+  h->dtype = p->dtype;
+  h->eps = p->ln_eps;
+  h->q_scale = tri::kLog2e / std::sqrt(static_cast<float>(kD));
+
+  std::vector<float> wq, wk, wv, wg, wb, wo, gamma, beta, bg, bo;
+  const tri_attn_dtype dt = p->dtype;
+  if ((rc = copy_to_host_f32(p->w_q, kHD * kCz, dt, wq, 0.f)) ||
+      (rc = copy_to_host_f32(p->w_k, kHD * kCz, dt, wk, 0.f)) ||
+      (rc = copy_to_host_f32(p->w_v, kHD * kCz, dt, wv, 0.f)) ||
+      (rc = copy_to_host_f32(p->w_g, kHD * kCz, dt, wg, 0.f)) ||
+      (rc = copy_to_host_f32(p->w_b, kHeads * kCz, dt, wb, 0.f)) ||
+      (rc = copy_to_host_f32(p->w_o, kCz * kHD, dt, wo, 0.f)) ||
+      (rc = copy_to_host_f32(p->ln_gamma, kCz, dt, gamma, 1.f)) ||
+      (rc = copy_to_host_f32(p->ln_beta, kCz, dt, beta, 0.f)) ||
+      (rc = copy_to_host_f32(p->b_g, kHD, dt, bg, 0.f)) ||
+      (rc = copy_to_host_f32(p->b_o, kCz, dt, bo, 0.f)))
+    return fail(rc);
+  for (float& x : wb) x *= tri::kLog2e;
+
+  if (dt == TRI_ATTN_BF16) {
+    // [Wq; Wk; Wv; Wg] as 512 K-major rows, and Wo as 128 K-major rows, both in the
+    // shared-memory image the tcgen05 B operand reads (bf16 bits kept exactly).
+    std::vector<uint16_t> w512(512 * 128), w128(128 * 128), img;
+    const std::vector<float>* parts[4] = {&wq, &wk, &wv, &wg};
+    for (int part = 0; part < 4; ++part)
+      for (int n = 0; n < kHD; ++n)
+        for (int c = 0; c < kCz; ++c)
+          w512[(part * kHD + n) * 128 + c] = f32_to_bf16_bits((*parts[part])[n * kCz + c]);
+    for (int n = 0; n < kCz; ++n)
+      for (int c = 0; c < kHD; ++c) w128[n * 128 + c] = f32_to_bf16_bits(wo[n * kHD + c]);
+    pack_kmajor_sw128(w512, 512, img);
+    if ((rc = upload(img, &h->w_qkvg))) return fail(rc);
+    pack_kmajor_sw128(w128, 128, img);
+    if ((rc = upload(img, &h->w_o))) return fail(rc);
+  } else {
+    std::vector<float> w512(512 * 128);
+    std::memcpy(&w512[0], wq.data(), kHD * kCz * 4);
+    std::memcpy(&w512[kHD * kCz], wk.data(), kHD * kCz * 4);
+    std::memcpy(&w512[2 * kHD * kCz], wv.data(), kHD * kCz * 4);
+    std::memcpy(&w512[3 * kHD * kCz], wg.data(), kHD * kCz * 4);
+    if ((rc = upload(w512, &h->w_qkvg))) return fail(rc);
+    if ((rc = upload(wo, &h->w_o))) return fail(rc);
+  }
+  void* tmp = nullptr;
+  if ((rc = upload(wb, &tmp))) return fail(rc);
+  h->w_b = static_cast<float*>(tmp);
+  if ((rc = upload(gamma, &tmp))) return fail(rc);
+  h->gamma = static_cast<float*>(tmp);
+  if ((rc = upload(beta, &tmp))) return fail(rc);
+  h->beta = static_cast<float*>(tmp);
+  if ((rc = upload(bg, &tmp))) return fail(rc);
+  h->b_g = static_cast<float*>(tmp);
+  if ((rc = upload(bo, &tmp))) return fail(rc);
+  h->b_o = static_cast<float*>(tmp);
+  if (cudaMalloc(&h->status, sizeof(int)) != cudaSuccess) return fail(TRI_ATTN_ERR_OOM);
+  if (cudaMemset(h->status, 0, sizeof(int)) != cudaSuccess) return fail(TRI_ATTN_ERR_CUDA);
+  *out = h;
+  return TRI_ATTN_OK;
+}
+
+int tri_attn_forward(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask,
+                     tri_attn_orientation orientation, void* out, void* stream, unsigned flags) {
+  if (!h || !Z || !out || N < 1) return TRI_ATTN_ERR_INVALID_ARG;
+  if (orientation != TRI_ATTN_STARTING && orientation != TRI_ATTN_ENDING)
+    return TRI_ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(Z) & 15) || (reinterpret_cast<uintptr_t>(out) & 15))
+    return TRI_ATTN_ERR_INVALID_ARG;
+  if (N > 46340) return TRI_ATTN_ERR_UNSUPPORTED;  // N*N pairs must fit in int32 per row index math
+  const size_t bytes = static_cast<size_t>(N) * N * kCz * esize(h->dtype);
+  if (Z != out && ranges_overlap(Z, out, bytes)) return TRI_ATTN_ERR_ALIAS;
+  if (cudaSetDevice(h->device) != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int rc = forward_impl(h, Z, N, mask, static_cast<int>(orientation), out, st, flags);
+  if (rc != TRI_ATTN_OK) return rc;
+  if (flags & TRI_ATTN_FLAG_SYNC) {
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+    return read_status(h, st);
+  }
+  return TRI_ATTN_OK;
+}
+
+int tri_attn_forward_host(tri_attn_handle* h, const void* Z_host, int N, const uint8_t* mask_host,
+                          const int* orientations, int n_orientations, void* out_host,
+                          void* stream, unsigned flags) {
+  if (!h || !Z_host || !out_host || N < 1 || n_orientations < 0 ||
+      (n_orientations > 0 && !orientations))
+    return TRI_ATTN_ERR_INVALID_ARG;
+  for (int t = 0; t < n_orientations; ++t)
+    if (orientations[t] != TRI_ATTN_STARTING && orientations[t] != TRI_ATTN_ENDING)
+      return TRI_ATTN_ERR_INVALID_ARG;
+  if (N > 46340) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (cudaSetDevice(h->device) != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(N) * N * kCz * esize(h->dtype);
+  if (h->stage_bytes < bytes) {
+    if (h->stage) cudaFree(h->stage);
+    h->stage = nullptr;
+    h->stage_bytes = 0;
+    CUDA_TRY(cudaMalloc(&h->stage, bytes));
+    h->stage_bytes = bytes;
+  }
+  const uint8_t* dmask = nullptr;
+  if (mask_host) {
+    if (h->stage_mask_bytes < static_cast<size_t>(N)) {
+      if (h->stage_mask) cudaFree(h->stage_mask);
+      h->stage_mask = nullptr;
+      h->stage_mask_bytes = 0;
+      CUDA_TRY(cudaMalloc(&h->stage_mask, static_cast<size_t>(N)));
+      h->stage_mask_bytes = N;
+    }
+    CUDA_TRY(cudaMemcpyAsync(h->stage_mask, mask_host, N, cudaMemcpyHostToDevice, st));
+    dmask = h->stage_mask;
+  }
+  CUDA_TRY(cudaMemcpyAsync(h->stage, Z_host, bytes, cudaMemcpyHostToDevice, st));
+  for (int t = 0; t < n_orientations; ++t) {
+    int rc = forward_impl(h, h->stage, N, dmask, orientations[t], h->stage, st,
+                          flags & ~TRI_ATTN_FLAG_SYNC);
+    if (rc != TRI_ATTN_OK) return rc;
+  }
+  CUDA_TRY(cudaMemcpyAsync(out_host, h->stage, bytes, cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaStreamSynchronize(st));
+  return read_status(h, st);
+}
+
+int tri_attn_get_status(tri_attn_handle* h, void* stream) {
+  if (!h) return TRI_ATTN_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+  return read_status(h, static_cast<cudaStream_t>(stream));
+}
+
+int tri_attn_kernel_times(tri_attn_handle* h, float ms[3], int launches[3]) {
+  if (!h || !ms) return TRI_ATTN_ERR_INVALID_ARG;
+  for (int k = 0; k < 3; ++k) {
+    float tot = 0.f;
+    for (int u = 0; u < h->ev_used[k]; ++u) {
+      float t = 0.f;
+      CUDA_TRY(cudaEventSynchronize(h->ev[k][u].b));
+      CUDA_TRY(cudaEventElapsedTime(&t, h->ev[k][u].a, h->ev[k][u].b));
+      tot += t;
+    }
+    ms[k] = tot;
+    if (launches) launches[k] = h->ev_used[k];
+    h->ev_used[k] = 0;
+  }
+  return TRI_ATTN_OK;
+}
+
+int tri_attn_set_workspace_limit(tri_attn_handle* h, size_t bytes) {
+  if (!h) return TRI_ATTN_ERR_INVALID_ARG;
+  h->ws_limit = bytes ? bytes : kDefaultWorkspaceLimit;
+  return TRI_ATTN_OK;
+}
+
+int tri_attn_debug_workspace(tri_attn_handle* h, void** q, void** k, void** v, void** g,
+                             void** bias, void** o, int* ld_bias, int* rows) {
+  if (!h) return TRI_ATTN_ERR_INVALID_ARG;
+  if (q) *q = h->q;
+  if (k) *k = h->k;
+  if (v) *v = h->v;
+  if (g) *g = h->g;
+  if (bias) *bias = h->bias;
+  if (o) *o = h->o;
+  if (ld_bias) *ld_bias = h->ld_bias;
+  if (rows) *rows = h->rows_last;
+  return TRI_ATTN_OK;
+}
+
+int tri_attn_destroy(tri_attn_handle* h) {
+  if (!h) return TRI_ATTN_OK;
+  cudaSetDevice(h->device);
+  void* ptrs[] = {h->w_qkvg, h->w_o, h->w_b, h->gamma, h->beta, h->b_g,
+                  h->b_o,    h->status, h->ws, h->stage, h->stage_mask};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+  for (auto& vec : h->ev)
+    for (auto& p : vec) {
+      if (p.a) cudaEventDestroy(p.a);
+      if (p.b) cudaEventDestroy(p.b);
+    }
+  delete h;
+  return TRI_ATTN_OK;
+}
+
+}  // extern "C"

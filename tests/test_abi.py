@@ -1,0 +1,92 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/tri_attn.h declares, and rejects bad arguments before
+touching a device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+from protein_pair_representation_layernorm_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_library_exports_every_declared_function():
+    L = binding.lib()
+    declared = binding.declared_functions()
+    assert len(declared) >= 9
+    for name in declared:
+        assert hasattr(L, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (tri_attn_\w+)", out))
+    assert set(declared) <= exported
+
+
+def test_status_strings():
+    for code in range(0, -8, -1):
+        s = binding.tri_attn_status_string(code)
+        assert s and s != "unknown status"
+    assert binding.tri_attn_status_string(-99) == "unknown status"
+
+
+def test_workspace_bytes():
+    ws = binding.tri_attn_workspace_bytes
+    assert ws(binding.TRI_ATTN_BF16, 0) == 0
+    assert ws(7, 10) == 0
+    # bf16: q, k, v, g, o (N*N*128 each) + bias H*N*roundup(N,64), 2 bytes per element
+    N = 1536
+    assert ws(binding.TRI_ATTN_BF16, N) >= 5 * N * N * 128 * 2 + 4 * N * N * 2
+    assert ws(binding.TRI_ATTN_F32, N) == 2 * ws(binding.TRI_ATTN_BF16, N)
+    assert ws(binding.TRI_ATTN_BF16, 4096) > ws(binding.TRI_ATTN_BF16, 1536)
+
+
+def test_create_rejects_bad_params_without_device():
+    L = binding.lib()
+    h = ctypes.c_void_p()
+    assert L.tri_attn_create(None, ctypes.byref(h)) == binding.TRI_ATTN_ERR_INVALID_ARG
+    p = binding.tri_attn_params()
+    p.c_z, p.n_heads, p.head_dim, p.dtype, p.ln_eps = 64, 4, 32, binding.TRI_ATTN_BF16, 1e-5
+    assert L.tri_attn_create(ctypes.byref(p), ctypes.byref(h)) == binding.TRI_ATTN_ERR_UNSUPPORTED
+    p.c_z = 128
+    # weight pointers missing
+    assert L.tri_attn_create(ctypes.byref(p), ctypes.byref(h)) == binding.TRI_ATTN_ERR_INVALID_ARG
+    p.dtype = 5
+    assert L.tri_attn_create(ctypes.byref(p), ctypes.byref(h)) == binding.TRI_ATTN_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
+def test_no_device_fails_loudly():
+    L = binding.lib()
+    p = binding.tri_attn_params()
+    p.c_z, p.n_heads, p.head_dim, p.dtype, p.ln_eps = 128, 4, 32, binding.TRI_ATTN_BF16, 1e-5
+    fake = ctypes.c_void_p(0x1000)
+    for f in ("ln_gamma", "ln_beta", "w_q", "w_k", "w_v", "w_g", "w_b", "w_o"):
+        setattr(p, f, fake.value)
+    h = ctypes.c_void_p()
+    assert L.tri_attn_create(ctypes.byref(p), ctypes.byref(h)) == binding.TRI_ATTN_ERR_NO_DEVICE
+    with pytest.raises(binding.TriAttnError):
+        binding.tri_attn_create(p)
+
+
+def test_null_handle_calls():
+    L = binding.lib()
+    assert L.tri_attn_forward(None, None, 1, None, 0, None, None, 0) == binding.TRI_ATTN_ERR_INVALID_ARG
+    assert L.tri_attn_get_status(None, None) == binding.TRI_ATTN_ERR_INVALID_ARG
+    assert L.tri_attn_destroy(None) == binding.TRI_ATTN_OK
+    assert L.tri_attn_set_workspace_limit(None, 0) == binding.TRI_ATTN_ERR_INVALID_ARG
+
+
+def test_product_path_never_touches_the_oracle():
+    """The package (kernels, binding, workloads) must not import, load or call oracle/."""
+    pkg = os.path.join(ROOT, "protein_pair_representation_layernorm_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
+                assert "liboracle" not in text, f
+                assert "oracle.c" not in text, f
