@@ -207,6 +207,13 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                   taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -239,6 +246,35 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for two values on the FMA pipe (x <= 64; results below 2^-126 flush to 0,
+// x = -inf gives exactly 0).  Cody-Waite style reduction x = n + f with
+// n = round(x), |f| <= 1/2: n is read from the low mantissa bits of x + 1.5 * 2^23.
+// 2^f is a degree-3 polynomial whose coefficients were fitted for minimal
+// relative error on [-1/2, 1/2] (iteratively reweighted least squares, max
+// relative error 7.5e-5); 2^n is applied by adding n to the exponent field, and
+// a result whose exponent would underflow (the sum turns negative) is clamped to 0.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const float2 xc = make_float2(fmaxf(x.x, -127.0f), fmaxf(x.y, -127.0f));
+  const float2 t = __fadd2_rn(xc, make_float2(kRound, kRound));
+  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), xc);
+  float2 p = __ffma2_rn(f, make_float2(0.05517132f, 0.05517132f),
+                        make_float2(0.24261054f, 0.24261054f));
+  p = __ffma2_rn(p, f, make_float2(0.69326097f, 0.69326097f));
+  p = __ffma2_rn(p, f, make_float2(0.99992812f, 0.99992812f));
+  const int a = max(__float_as_int(p.x) + (__float_as_int(t.x) << 23), 0);
+  const int b = max(__float_as_int(p.y) + (__float_as_int(t.y) << 23), 0);
+  return make_float2(__int_as_float(a), __int_as_float(b));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -10,7 +10,7 @@
 // before any attention runs; when the workspace for all rows exceeds the
 // handle's limit, a bias-only pass runs first and the rest proceeds in row
 // chunks.
-#include "../../include/tri_attn.h"
+#include "tri_attn.h"
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -167,6 +167,12 @@ int set_kernel_attrs() {
                                 tri::attn::kSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(tri::gout::kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 tri::gout::kSmemBytes));
+  if (log_enabled()) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, tri::attn::kernel) == cudaSuccess)
+      TA_LOG("tri_attn_fwd: regs %d, max threads %d, static smem %zu, local %zu", fa.numRegs,
+             fa.maxThreadsPerBlock, fa.sharedSizeBytes, fa.localSizeBytes);
+  }
   attrs_set = true;
   return TRI_ATTN_OK;
 }
@@ -431,11 +437,12 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
     const unsigned grid = static_cast<unsigned>(std::min<long long>(ntiles, h->num_sms));
     Timer tm(h, st, timed, 0);
     tri::plp::kernel<<<grid, tri::plp::kThreads, tri::plp::kSmemBytes, st>>>(a);
+    return cudaGetLastError();
   };
-  if (chunked) proj(0, N, 0, 1);
+  if (chunked) CUDA_TRY(proj(0, N, 0, 1));
   for (int r0 = 0; r0 < N; r0 += rows) {
     const int nr = std::min(rows, N - r0);
-    proj(r0, nr, 1, chunked ? 0 : 1);
+    CUDA_TRY(proj(r0, nr, 1, chunked ? 0 : 1));
     {
       CUtensorMap mq, mk, mv, mb;
       const uint64_t rh = static_cast<uint64_t>(nr) * kHeads;
@@ -460,6 +467,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
       Timer tm(h, st, timed, 1);
       tri::attn::kernel<<<grid, tri::attn::kThreads, tri::attn::kSmemBytes, st>>>(mq, mk, mv, mb,
                                                                                  a);
+      CUDA_TRY(cudaGetLastError());
     }
     {
       tri::GateArgs a{};
@@ -477,6 +485,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
       dim3 grid(jtiles, nr);
       Timer tm(h, st, timed, 2);
       tri::gout::kernel<<<grid, tri::gout::kThreads, tri::gout::kSmemBytes, st>>>(a);
+      CUDA_TRY(cudaGetLastError());
     }
   }
   h->rows_last = N - (N - 1) / rows * rows;

@@ -14,17 +14,25 @@
 // The 4 rows share every bias tile b_h(j0.., k-tile), which is loaded once per
 // CTA; K and V differ per row.
 //
-// Warp roles (320 threads):
-//   warps 0-3  softmax group 0: rows i0, i0+1   (thread = query j, TMEM lane j)
-//   warps 4-7  softmax group 1: rows i0+2, i0+3
-//   warp 8     TMA producer: Q once; per key tile K, V of the 4 rows + the bias tile
-//   warp 9     MMA issuer (one thread): S_r = Q_r K_r^T (M=128, N=64, K=32),
-//              O_r += P_r V_r (M=128, N=32, K=64, P read from TMEM)
+// Warp roles (576 threads):
+//   warps 4r..4r+3  softmax group r = row i0+r (thread = query j = TMEM lane j)
+//   warp 16         TMA producer: Q once; per key tile K, V of the 4 rows + the bias tile
+//   warp 17         MMA issuer (one thread): S_r = Q_r K_r^T (M=128, N=64, K=32),
+//                   O_r += P_r V_r (M=128, N=32, K=64, P read from TMEM)
 // TMEM (512 columns): S_r/P_r at columns 64r (fp32 scores, bf16 P aliased over
 // the first 32 columns), O_r at 256 + 32r.
 // Pipeline: 3 shared-memory stages of {K[4][64][32], V[4][64][32], bias[128][64]}.
-// The two softmax groups alternate with the tensor core: while one group
-// turns S into P, the MMA warp runs the other group's PV and next QK.
+// The four softmax groups interleave with the tensor core: while a group turns
+// its S into P, the MMA warp runs the other groups' PV and next QK.
+//
+// The exponentials are the binding resource (the special-function unit does 16
+// per clock per SM, against 8192 MMA flops; at d = 32 each score needs one
+// exponential per 128 flops).  A compile-time fraction of them (kEmuEvery) is
+// evaluated on the FMA pipe instead: 2^x = 2^n * 2^f with n = round(x) (Cody-Waite
+// range reduction, n obtained by the 1.5 * 2^23 rounding constant) and 2^f, |f| <= 1/2,
+// from a degree-3 polynomial fitted here for minimal relative error (7.5e-5, below
+// the 2^-9 of the bf16 P it feeds); 2^n is applied by adding n to the exponent
+// field of the polynomial value.
 //
 // Online softmax per (row, query): the running offset m is raised only when a
 // tile's maximum exceeds it by more than kTau (log2 units), so the O rescale in
@@ -45,11 +53,17 @@ namespace attn {
 constexpr int kBJ = 128;          // queries per CTA
 constexpr int kBK = 64;           // keys per step
 constexpr int kRows = 4;          // problem rows per CTA
-constexpr int kGroups = 2;        // softmax warpgroups (2 rows each)
+constexpr int kGroups = 4;        // softmax warpgroups, one row each
 constexpr int kStages = 3;
-constexpr int kThreads = 320;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+// 18 warps: 16 softmax + producer + MMA issuer.  Five of them share one SM
+// sub-partition (16K registers), which caps the kernel at 96 registers per thread.
+constexpr int kThreads = (4 * kGroups + 2) * 32;
+constexpr int kProducerWarp = 4 * kGroups;
+constexpr int kMmaWarp = 4 * kGroups + 1;
+#ifndef TRI_ATTN_EMU_EVERY
+#define TRI_ATTN_EMU_EVERY 0
+#endif
+constexpr int kEmuEvery = TRI_ATTN_EMU_EVERY;  // every kEmuEvery-th pair of scores: FMA exp2
 constexpr float kTau = 8.0f;
 constexpr float kFloor = -1.0e30f;
 
@@ -172,17 +186,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sSt = smem_u32(smem + kSmemStages);
       bool ok = mbar_wait(q_full, 0, abort_flag);
       bool issued = false;
-      auto issue_pv = [&](int g, int tt) {
+      auto issue_pv = [&](int r, int tt) {
         const uint32_t sV = sSt + (tt % kStages) * kStageBytes + kStageV;
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const int r = 2 * g + rr;
-#pragma unroll
-          for (int kc = 0; kc < kBK / 16; ++kc) {
-            const uint64_t bd = smem_desc(sV + r * kKVTileBytes + kc * 1024, 512, kSwizzle64B);
-            mma_ts(tmem + kColO + 32 * r, tmem + kColS + 64 * r + kc * 8, bd, kIdescPV,
-                   (tt > 0 || kc > 0) ? 1u : 0u);
-          }
+        for (int kc = 0; kc < kBK / 16; ++kc) {
+          const uint64_t bd = smem_desc(sV + r * kKVTileBytes + kc * 1024, 512, kSwizzle64B);
+          mma_ts(tmem + kColO + 32 * r, tmem + kColS + 64 * r + kc * 8, bd, kIdescPV,
+                 (tt > 0 || kc > 0) ? 1u : 0u);
         }
       };
       for (int t = 0; ok && t < T; ++t) {
@@ -197,14 +207,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_pv(g, t - 1);
           }
 #pragma unroll
-          for (int rr = 0; rr < 2; ++rr) {
-            const int r = 2 * g + rr;
-#pragma unroll
-            for (int kc = 0; kc < kD / 16; ++kc) {
-              const uint64_t ad = smem_desc(sQ + r * kQTileBytes + kc * 32, 512, kSwizzle64B);
-              const uint64_t bd = smem_desc(sK + r * kKVTileBytes + kc * 32, 512, kSwizzle64B);
-              mma_ss(tmem + kColS + 64 * r, ad, bd, kIdescQK, kc > 0 ? 1u : 0u);
-            }
+          for (int kc = 0; kc < kD / 16; ++kc) {
+            const uint64_t ad = smem_desc(sQ + g * kQTileBytes + kc * 32, 512, kSwizzle64B);
+            const uint64_t bd = smem_desc(sK + g * kKVTileBytes + kc * 32, 512, kSwizzle64B);
+            mma_ss(tmem + kColS + 64 * g, ad, bd, kIdescQK, kc > 0 ? 1u : 0u);
           }
           issued = true;
           mma_commit(&s_full[g]);
@@ -232,14 +238,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp < kProducerWarp) {
     // ------------------------------------------------------------ softmax
-    const int g = warp >> 2;              // softmax group
+    const int g = warp >> 2;              // softmax group = row of the CTA
     const int quad = warp & 3;            // TMEM lane quadrant
     const int jl = quad * 32 + lane;      // query within the tile
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    float m_used[2] = {kFloor, kFloor};
-    float l_sum[2] = {0.f, 0.f};
+    const uint32_t colS = tmem + lane_base + kColS + 64 * g;
+    const uint32_t colO = tmem + lane_base + kColO + 32 * g;
+    float m_used = kFloor;
+    float l_sum = 0.f;
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       const int s = t % kStages;
@@ -250,65 +258,76 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      // bias row jl of this key tile: 64 bf16 in 128-byte swizzled rows
+      // x = s + b (base-2 logits) in two 32-key halves; tile maximum over four
+      // independent chains.  The bias row jl of this key tile is 64 bf16 in a
+      // 128-byte swizzled row: 16-byte chunk c sits at position c ^ (jl % 8).
       const uint8_t* brow = smem + kSmemStages + s * kStageBytes + kStageB + jl * 128;
-      uint32_t bw[32];
+      float2 x[32];
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4*>(brow + ((c ^ (jl & 7)) << 4));
-        bw[4 * c] = v.x;
-        bw[4 * c + 1] = v.y;
-        bw[4 * c + 2] = v.z;
-        bw[4 * c + 3] = v.w;
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sr[32];
+        tmem_ld32(colS + 32 * half, sr);
+        uint32_t bw[16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 v =
+              *reinterpret_cast<const uint4*>(brow + (((half * 4 + c) ^ (jl & 7)) << 4));
+          bw[4 * c] = v.x;
+          bw[4 * c + 1] = v.y;
+          bw[4 * c + 2] = v.z;
+          bw[4 * c + 3] = v.w;
+        }
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float2& xe = x[half * 16 + e];
+          xe = __fadd2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
+                          make_float2(bf16lo_to_f32(bw[e]), bf16hi_to_f32(bw[e])));
+          mx[e & 3] = fmax3(mx[e & 3], xe.x, xe.y);
+        }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&st_empty[s]);
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int r = 2 * g + rr;
-        const uint32_t colS = tmem + lane_base + kColS + 64 * r;
-        uint32_t sr[64];
-        tmem_ld32(colS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(colS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_ld_wait();
-        float x[64];
-        float tmax = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          x[2 * e] = __uint_as_float(sr[2 * e]) + bf16lo_to_f32(bw[e]);
-          x[2 * e + 1] = __uint_as_float(sr[2 * e + 1]) + bf16hi_to_f32(bw[e]);
-          tmax = fmaxf(tmax, fmaxf(x[2 * e], x[2 * e + 1]));
-        }
-        const float m_new = fmaxf(m_used[rr], tmax);
-        const bool need = m_new > m_used[rr] + kTau;
-        float scale = 1.0f;
-        if (need) {
-          scale = ex2_approx(m_used[rr] - m_new);
-          l_sum[rr] *= scale;
-          m_used[rr] = m_new;
-        }
-        if (t > 0 && __any_sync(0xffffffffu, need)) {
-          const uint32_t colO = tmem + lane_base + kColO + 32 * r;
-          uint32_t ov[32];
-          tmem_ld32(colO, ov);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * scale);
-          tmem_st32(colO, ov);
-        }
-        const float mu = m_used[rr];
-        float lsum = 0.f;
-        uint32_t pk[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float p0 = ex2_approx(x[2 * e] - mu);
-          const float p1 = ex2_approx(x[2 * e + 1] - mu);
-          lsum += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
-        }
-        l_sum[rr] += lsum;
-        tmem_st32(colS, pk);
+      if (lane == 0) mbar_arrive(&st_empty[s]);  // this warp is done with the bias tile
+      const float tmax = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+      // lazy rescale: raise the offset only when the tile max exceeds it by > kTau
+      const bool need = tmax > m_used + kTau;
+      float scale = 1.0f;
+      if (need) {
+        scale = ex2_approx(m_used - tmax);
+        l_sum *= scale;
+        m_used = tmax;
       }
+      if (t > 0 && __any_sync(0xffffffffu, need)) {
+        uint32_t ov[32];
+        tmem_ld32(colO, ov);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * scale);
+        tmem_st32(colO, ov);
+      }
+      const float2 neg_m = make_float2(-m_used, -m_used);
+      float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int quarter = 0; quarter < 4; ++quarter) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int e = quarter * 8 + q;
+          const float2 dlt = __fadd2_rn(x[e], neg_m);
+          float2 p;
+          if (kEmuEvery > 0 && (e % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1) {
+            p = exp2_poly2(dlt);
+          } else {
+            p = make_float2(ex2_approx(dlt.x), ex2_approx(dlt.y));
+          }
+          acc[e & 1] = __fadd2_rn(acc[e & 1], p);
+          pk[q] = pack_bf16x2(p.x, p.y);
+        }
+        tmem_st8(colS + 8 * quarter, pk);
+      }
+      const float2 a = __fadd2_rn(acc[0], acc[1]);
+      l_sum += a.x + a.y;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -319,26 +338,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       const int j = j0 + jl;
+      const int row = ig * kRows + g;
+      uint32_t ov[32];
+      tmem_ld32(colO, ov);
+      tmem_ld_wait();
+      if (row < a.rows && j < a.N) {
+        const float inv = l_sum > 0.f ? 1.0f / l_sum : 0.f;
+        uint32_t pk[16];
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int r = 2 * g + rr;
-        const int row = ig * kRows + r;
-        uint32_t ov[32];
-        tmem_ld32(tmem + lane_base + kColO + 32 * r, ov);
-        tmem_ld_wait();
-        if (row < a.rows && j < a.N) {
-          const float inv = l_sum[rr] > 0.f ? 1.0f / l_sum[rr] : 0.f;
-          uint32_t pk[16];
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
+        uint4* dst = reinterpret_cast<uint4*>(
+            a.O + ((static_cast<long long>(row) * kHeads + h) * a.N + j) * kD);
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv,
-                                __uint_as_float(ov[2 * e + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(
-              a.O + ((static_cast<long long>(row) * kHeads + h) * a.N + j) * kD);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        }
+        for (int q = 0; q < 4; ++q)
+          dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       }
     } else if (lane == 0) {
       *abort_flag = 1;
