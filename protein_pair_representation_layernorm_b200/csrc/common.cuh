@@ -13,6 +13,11 @@ constexpr int kHeads = 4;       // attention heads
 constexpr int kD = 32;          // head width
 constexpr int kHD = kHeads * kD;
 constexpr float kLog2e = 1.4426950408889634f;
+// Logit bias of a masked (or padding) key in the bf16 path.  Finite on purpose:
+// the attention kernel adds the bias with an identity-matrix MMA, where the
+// zeros of the identity meet every bias entry of the tile, and 0 * (-inf) would
+// be NaN.  2^(kMaskedLogit - m) is exactly 0 in fp32 for any finite offset m.
+constexpr float kMaskedLogit = -3.0e38f;
 
 // Offset (in elements) of pair (i, j) of the problem inside Z / out.  The
 // ending-node block reads and writes the pair representation through the

@@ -33,7 +33,7 @@ constexpr uint32_t kSmemBar = kSmemBo + kCz * 4;
 constexpr uint32_t kSmemBytes = kSmemBar + 64 + 1024;
 constexpr uint32_t kTmemCols = 128;
 
-__global__ void __launch_bounds__(kThreads) kernel(const GateArgs a) {
+__global__ void __launch_bounds__(kThreads) gate_out(const GateArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));

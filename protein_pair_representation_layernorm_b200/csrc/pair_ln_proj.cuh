@@ -5,8 +5,8 @@
 // row (pairs (i, j0..j0+127)).  Thread t owns pair j0+t:
 //   1. reads its 256-byte pair vector (the ending-node block reads Z[j][i]),
 //   2. LayerNorm in fp32 (mean, biased variance, rsqrt),
-//   3. the per-head logit bias  Wb x  in fp32 (Wb pre-scaled by log2 e; -inf at
-//      masked keys and at the padding columns j >= N),
+//   3. the per-head logit bias  Wb x  in fp32 (Wb pre-scaled by log2 e;
+//      kMaskedLogit at masked keys and at the padding columns j >= N),
 //   4. writes x as bf16 into the MMA A tile in shared memory (K-major, 128-byte
 //      swizzle).
 // Thread 0 then issues 16 tcgen05 MMAs, D[128 x 512] = X[128 x 128] W^T, where
@@ -39,7 +39,7 @@ constexpr uint32_t kSmemBar = kSmemPar + kParFloats * 4;
 constexpr uint32_t kSmemBytes = kSmemBar + 64 + 1024;         // + alignment slack
 constexpr uint32_t kTmemCols = 512;
 
-__global__ void __launch_bounds__(kThreads, 1) kernel(const ProjArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1) kernel(const ProjArgs a) {
 #pragma unroll
         for (int h = 0; h < kHeads; ++h)
           a.bias[(static_cast<long long>(h) * a.N + i) * a.ld_bias + j] =
-              __float2bfloat16_rn(key_valid ? bacc[h] : -INFINITY);
+              __float2bfloat16_rn(key_valid ? bacc[h] : kMaskedLogit);
       }
     }
     if (!qkvg) continue;

@@ -161,15 +161,15 @@ bool attrs_set = false;
 
 int set_kernel_attrs() {
   if (attrs_set) return TRI_ATTN_OK;
-  CUDA_TRY(cudaFuncSetAttribute(tri::plp::kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  CUDA_TRY(cudaFuncSetAttribute(tri::plp::pair_ln_proj, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 tri::plp::kSmemBytes));
-  CUDA_TRY(cudaFuncSetAttribute(tri::attn::kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  CUDA_TRY(cudaFuncSetAttribute(tri::attn::tri_attn_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 tri::attn::kSmemBytes));
-  CUDA_TRY(cudaFuncSetAttribute(tri::gout::kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  CUDA_TRY(cudaFuncSetAttribute(tri::gout::gate_out, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 tri::gout::kSmemBytes));
   if (log_enabled()) {
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, tri::attn::kernel) == cudaSuccess)
+    if (cudaFuncGetAttributes(&fa, tri::attn::tri_attn_fwd) == cudaSuccess)
       TA_LOG("tri_attn_fwd: regs %d, max threads %d, static smem %zu, local %zu", fa.numRegs,
              fa.maxThreadsPerBlock, fa.sharedSizeBytes, fa.localSizeBytes);
   }
@@ -436,7 +436,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
     const long long ntiles = static_cast<long long>(nrows) * jtiles;
     const unsigned grid = static_cast<unsigned>(std::min<long long>(ntiles, h->num_sms));
     Timer tm(h, st, timed, 0);
-    tri::plp::kernel<<<grid, tri::plp::kThreads, tri::plp::kSmemBytes, st>>>(a);
+    tri::plp::pair_ln_proj<<<grid, tri::plp::kThreads, tri::plp::kSmemBytes, st>>>(a);
     return cudaGetLastError();
   };
   if (chunked) CUDA_TRY(proj(0, N, 0, 1));
@@ -465,7 +465,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
       a.status = h->status;
       dim3 grid(jtiles, (nr + tri::attn::kRows - 1) / tri::attn::kRows, kHeads);
       Timer tm(h, st, timed, 1);
-      tri::attn::kernel<<<grid, tri::attn::kThreads, tri::attn::kSmemBytes, st>>>(mq, mk, mv, mb,
+      tri::attn::tri_attn_fwd<<<grid, tri::attn::kThreads, tri::attn::kSmemBytes, st>>>(mq, mk, mv, mb,
                                                                                  a);
       CUDA_TRY(cudaGetLastError());
     }
@@ -484,7 +484,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
       a.status = h->status;
       dim3 grid(jtiles, nr);
       Timer tm(h, st, timed, 2);
-      tri::gout::kernel<<<grid, tri::gout::kThreads, tri::gout::kSmemBytes, st>>>(a);
+      tri::gout::gate_out<<<grid, tri::gout::kThreads, tri::gout::kSmemBytes, st>>>(a);
       CUDA_TRY(cudaGetLastError());
     }
   }

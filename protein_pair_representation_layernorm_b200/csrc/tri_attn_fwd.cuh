@@ -88,7 +88,7 @@ struct Maps {
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
-    kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+    tri_attn_fwd(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
            const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_b,
            const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
