@@ -6,8 +6,9 @@
 // by pair_ln_proj, o = attention output of the 4 heads), rounds it to bf16 and
 // writes it into the MMA A tile (K-major, 128-byte swizzle).  Thread 0 issues 8
 // tcgen05 MMAs, D[128 x 128] = (G*O) Wo^T, fp32 in 128 TMEM columns; each
-// thread then adds bo and its own residual z_ij and writes out_ij as bf16 with
-// 16-byte vector stores.  The ending-node block reads the residual from and
+// thread then adds bo and its own residual z_ij (loaded at the start, together
+// with o and g, so that all of a thread's loads are in flight at once) and writes
+// out_ij as bf16 with 16-byte vector stores.  The ending-node block reads the residual from and
 // writes the result to the swapped view (pair (i, j) is Z[j][i]).  A thread
 // reads z_ij before writing out_ij, so out may alias Z.
 //
@@ -71,6 +72,15 @@ __global__ void __launch_bounds__(kThreads) gate_out(const GateArgs a) {
   const int j = blockIdx.x * kTileM + tid;
   const bool jv = j < a.N;
 
+  // ---- the residual pair vector: loaded now so that it is in flight with o and g
+  const long long zoff = jv ? pair_offset(a.orient, a.N, i, j) : 0;
+  uint4 zv[16];
+  if (jv) {
+    const uint4* zp = reinterpret_cast<const uint4*>(a.Z + zoff);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) zv[q] = zp[q];
+  }
+
   // ---- A = bf16(g * o), K index = h*d + e
 #pragma unroll
   for (int h = 0; h < kHeads; ++h) {
@@ -131,21 +141,17 @@ __global__ void __launch_bounds__(kThreads) gate_out(const GateArgs a) {
   if (__syncthreads_and(done ? 1 : 0)) {
     tc_fence_after();
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const long long zoff = jv ? pair_offset(a.orient, a.N, i, j) : 0;
-#pragma unroll 1
+#pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
       uint32_t v[32];
       tmem_ld32(tmem + lane_base + cc * 32, v);
       tmem_ld_wait();
       if (!jv) continue;
-      const uint4* zp = reinterpret_cast<const uint4*>(a.Z + zoff + cc * 32);
-      uint4 zv[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) zv[q] = zp[q];
       uint32_t pk[16];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const uint32_t zw[4] = {zv[q].x, zv[q].y, zv[q].z, zv[q].w};
+        const uint4 zq = zv[cc * 4 + q];
+        const uint32_t zw[4] = {zq.x, zq.y, zq.z, zq.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int c0 = cc * 32 + q * 8 + 2 * e;

@@ -1,19 +1,22 @@
 // pair_ln_proj.cuh — LayerNorm + fused Q/K/V/gate projection (tcgen05) + logit
 // bias, bf16 pair representation.
 //
-// One CTA of 128 threads is persistent over tiles of 128 pairs of one problem
-// row (pairs (i, j0..j0+127)).  Thread t owns pair j0+t:
+// Persistent CTAs of two independent 128-thread groups.  Each group walks its
+// own tiles of 128 pairs of one problem row (pairs (i, j0..j0+127)); thread t of
+// the group owns pair j0+t:
 //   1. reads its 256-byte pair vector (the ending-node block reads Z[j][i]),
 //   2. LayerNorm in fp32 (mean, biased variance, rsqrt),
 //   3. the per-head logit bias  Wb x  in fp32 (Wb pre-scaled by log2 e;
 //      kMaskedLogit at masked keys and at the padding columns j >= N),
-//   4. writes x as bf16 into the MMA A tile in shared memory (K-major, 128-byte
-//      swizzle).
-// Thread 0 then issues 16 tcgen05 MMAs, D[128 x 512] = X[128 x 128] W^T, where
-// W = [Wq; Wk; Wv; Wg] stays resident in shared memory for the whole kernel,
-// accumulating in fp32 in all 512 TMEM columns.  Each thread reads back its
-// TMEM lane and writes q (scaled by log2(e)/sqrt(d)), k, v head-major
-// ([rows][H][N][d]) and sigmoid(g + bg) pair-major ([rows][N][H*d]), bf16.
+//   4. writes x as bf16 into the group's MMA A tile in shared memory (K-major,
+//      128-byte swizzle), then prefetches the pair vector of its next tile.
+// One thread of the group then issues the projection D = X W^T in two halves of
+// N = 256 (q|k, then v|g), W = [Wq; Wk; Wv; Wg] resident in shared memory for the
+// whole kernel, each half accumulating in fp32 in the group's 256 TMEM columns.
+// Each thread reads back its TMEM lane and writes q (scaled by log2(e)/sqrt(d)),
+// k, v head-major ([rows][H][N][d]) and sigmoid(g + bg) pair-major
+// ([rows][N][H*d]), bf16.  While one group runs its MMAs the other normalises or
+// stores, so the tensor core, the ALUs and HBM overlap.
 //
 // This is the HBM-bound step: per pair it reads 256 B and writes 1 KB + 8 B.
 #pragma once
@@ -24,7 +27,9 @@
 namespace tri {
 namespace plp {
 
-constexpr int kThreads = 128;
+constexpr int kGroupThreads = 128;
+constexpr int kGroupsPerCta = 2;
+constexpr int kThreads = kGroupThreads * kGroupsPerCta;
 constexpr int kTileM = 128;
 constexpr int kNOut = 4 * kHD;                       // q | k | v | g
 constexpr uint32_t kWImgBytes = kNOut * kCz * 2;     // 131072
@@ -32,30 +37,47 @@ constexpr uint32_t kWAtomBytes = kNOut * 128;        // one 64-element K slab of
 constexpr uint32_t kATileBytes = kTileM * kCz * 2;   // 32768
 constexpr uint32_t kAAtomBytes = kTileM * 128;       // 16384
 constexpr uint32_t kSmemW = 0;
-constexpr uint32_t kSmemA = kWImgBytes;
-constexpr uint32_t kSmemPar = kSmemA + kATileBytes;           // fp32 params
-constexpr uint32_t kParFloats = kHeads * kCz + 3 * kCz;       // w_b, gamma, beta, b_g
+constexpr uint32_t kSmemA = kWImgBytes;                                  // + grp * kATileBytes
+constexpr uint32_t kSmemPar = kSmemA + kGroupsPerCta * kATileBytes;     // fp32 params
+constexpr uint32_t kParFloats = kHeads * kCz + 3 * kCz;                 // w_b, gamma, beta, b_g
 constexpr uint32_t kSmemBar = kSmemPar + kParFloats * 4;
-constexpr uint32_t kSmemBytes = kSmemBar + 64 + 1024;         // + alignment slack
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSmemBytes = kSmemBar + 64 + 1024;                   // + alignment slack
+constexpr uint32_t kTmemCols = 512;                                     // 256 per group
+
+__device__ __forceinline__ void load_pair(const ProjArgs& a, long long tile, int jtiles, int gt,
+                                          uint4 (&zr)[16]) {
+  const int r = static_cast<int>(tile / jtiles);
+  const int j = static_cast<int>(tile % jtiles) * kTileM + gt;
+  if (j < a.N) {
+    const uint4* zp =
+        reinterpret_cast<const uint4*>(a.Z + pair_offset(a.orient, a.N, a.row0 + r, j));
+#pragma unroll
+    for (int c = 0; c < 16; ++c) zr[c] = __ldg(zp + c);
+  } else {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) zr[c] = make_uint4(0, 0, 0, 0);
+  }
+}
 
 __global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sW = smem + kSmemW;
-  uint8_t* sA = smem + kSmemA;
   float* s_wb = reinterpret_cast<float*>(smem + kSmemPar);
   float* s_gamma = s_wb + kHeads * kCz;
   float* s_beta = s_gamma + kCz;
   float* s_bg = s_beta + kCz;
   uint64_t* w_bar = reinterpret_cast<uint64_t*>(smem + kSmemBar);
-  uint64_t* mma_bar = w_bar + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(w_bar + 2);
+  uint64_t* mma_bar = w_bar + 1;  // one per group
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + kGroupsPerCta);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5;
+  const int grp = tid / kGroupThreads;
+  const int gt = tid % kGroupThreads;           // pair within the tile = TMEM lane
+  const uint32_t bar_id = 1 + grp;
   const bool qkvg = a.write_qkvg != 0;
+  uint8_t* sA = smem + kSmemA + grp * kATileBytes;
 
   for (int idx = tid; idx < kHeads * kCz; idx += kThreads) s_wb[idx] = a.w_b[idx];
   for (int idx = tid; idx < kCz; idx += kThreads) {
@@ -65,7 +87,7 @@ __global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
   }
   if (tid == 0) {
     mbar_init(w_bar, 1);
-    mbar_init(mma_bar, 1);
+    for (int g = 0; g < kGroupsPerCta; ++g) mbar_init(&mma_bar[g], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -76,40 +98,33 @@ __global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
+  const uint32_t tmem = *tmem_slot + static_cast<uint32_t>(grp * 256);
   if (tid == 0 && qkvg) {
     mbar_arrive_expect_tx(w_bar, kWImgBytes);
     for (uint32_t off = 0; off < kWImgBytes; off += 32768)
-      bulk_load(sW + off, a.w_img + off, 32768, w_bar);
+      bulk_load(smem + kSmemW + off, a.w_img + off, 32768, w_bar);
   }
 
   const int jtiles = (a.N + kTileM - 1) / kTileM;
   const long long ntiles = static_cast<long long>(a.rows) * jtiles;
-  const uint32_t sA_u32 = smem_u32(sA), sW_u32 = smem_u32(sW);
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  const long long stride = static_cast<long long>(gridDim.x) * kGroupsPerCta;
+  const uint32_t sA_u32 = smem_u32(sA), sW_u32 = smem_u32(smem + kSmemW);
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   constexpr uint32_t kIdesc = idesc_bf16_f32(128, 256, false);
   uint32_t mma_phase = 0;
   bool w_ready = false;
+  const bool mma_thread = gt == 0;
 
-  for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+  long long tile = static_cast<long long>(blockIdx.x) * kGroupsPerCta + grp;
+  uint4 zr[16];
+  if (tile < ntiles) load_pair(a, tile, jtiles, gt, zr);
+  for (; tile < ntiles; tile += stride) {
     const int r = static_cast<int>(tile / jtiles);
-    const int jt = static_cast<int>(tile % jtiles);
     const int i = a.row0 + r;
-    const int j = jt * kTileM + tid;
+    const int j = static_cast<int>(tile % jtiles) * kTileM + gt;
     const bool jv = j < a.N;
 
-    // ---- 1. pair vector (128 bf16 = 16 x 16 B)
-    uint4 zr[16];
-    if (jv) {
-      const uint4* zp = reinterpret_cast<const uint4*>(a.Z + pair_offset(a.orient, a.N, i, j));
-#pragma unroll
-      for (int c = 0; c < 16; ++c) zr[c] = __ldg(zp + c);
-    } else {
-#pragma unroll
-      for (int c = 0; c < 16; ++c) zr[c] = make_uint4(0, 0, 0, 0);
-    }
-    // ---- 2. LayerNorm statistics in fp32 (two passes over registers)
+    // ---- LayerNorm statistics in fp32 (two passes over registers)
     float sum = 0.f;
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
@@ -131,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
     }
     const float rstd = rsqrtf(var * (1.0f / kCz) + a.eps);
 
-    // ---- 3./4. normalise, bias dot products, bf16 A tile
+    // ---- normalise, bias dot products, bf16 A tile
     float bacc[kHeads] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
@@ -150,8 +165,8 @@ __global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
         packed[e] = pack_bf16x2(x0, x1);
       }
       if (qkvg) {
-        // K-major, 128 B swizzle: row tid, 16-byte chunk (c % 8) of K-slab c / 8
-        uint8_t* dst = sA + (c >> 3) * kAAtomBytes + tid * 128 + ((((c & 7) ^ (tid & 7))) << 4);
+        // K-major, 128 B swizzle: row gt, 16-byte chunk (c % 8) of K-slab c / 8
+        uint8_t* dst = sA + (c >> 3) * kAAtomBytes + gt * 128 + (((c & 7) ^ (gt & 7)) << 4);
         *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
       }
     }
@@ -164,96 +179,103 @@ __global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
               __float2bfloat16_rn(key_valid ? bacc[h] : kMaskedLogit);
       }
     }
+    // ---- prefetch the next tile's pair vector while this one is projected
+    if (tile + stride < ntiles) load_pair(a, tile + stride, jtiles, gt, zr);
     if (!qkvg) continue;
 
-    // ---- MMA: D[128 x 512] = X W^T
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    named_barrier_sync(bar_id, kGroupThreads);
     tc_fence_after();
-    if (tid == 0) {
-      bool ok = true;
-      if (!w_ready) {
-        ok = mbar_wait(w_bar, 0, abort_flag);
-        w_ready = ok;
-      }
-      if (ok) {
-#pragma unroll
-        for (int nh = 0; nh < 2; ++nh) {
+
+    bool ok = true;
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+      // ---- MMA: D[128 x 256] = X W[half*256 .. half*256+255]^T
+      if (mma_thread) {
+        bool ready = true;
+        if (!w_ready) {
+          ready = mbar_wait(w_bar, 0, abort_flag);
+          w_ready = ready;
+        }
+        if (ready) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint64_t ad = smem_desc(sA_u32 + (kk >> 2) * kAAtomBytes + (kk & 3) * 32, 1024,
                                           kSwizzle128B);
             const uint64_t bd = smem_desc(
-                sW_u32 + (kk >> 2) * kWAtomBytes + nh * 256 * 128 + (kk & 3) * 32, 1024,
+                sW_u32 + (kk >> 2) * kWAtomBytes + half * 256 * 128 + (kk & 3) * 32, 1024,
                 kSwizzle128B);
-            mma_ss(tmem + nh * 256, ad, bd, kIdesc, kk > 0 ? 1u : 0u);
+            mma_ss(tmem, ad, bd, kIdesc, kk > 0 ? 1u : 0u);
           }
+          mma_commit(&mma_bar[grp]);
+        } else {
+          *abort_flag = 1;
+          report_status(a.status, kStatusTimeout);
         }
-        mma_commit(mma_bar);
-      } else {
-        *abort_flag = 1;
-        report_status(a.status, kStatusTimeout);
       }
+      const bool done = mbar_wait(&mma_bar[grp], mma_phase, abort_flag);
+      mma_phase ^= 1;
+      if (!named_barrier_and(bar_id, kGroupThreads, done)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+
+      // ---- epilogue: TMEM lane gt -> two of q, k, v, g of pair j
+#pragma unroll 1
+      for (int cc = 0; cc < 8; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + cc * 32, v);
+        tmem_ld_wait();
+        if (!jv) continue;
+        const int part = half * 2 + (cc >> 2), h = cc & 3;
+        uint32_t pk[16];
+        if (part < 3) {
+          const float sc = part == 0 ? a.q_scale : 1.0f;
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
+          __nv_bfloat16* base = part == 0 ? a.Q : (part == 1 ? a.K : a.V);
+          uint4* dst = reinterpret_cast<uint4*>(
+              base + ((static_cast<long long>(r) * kHeads + h) * a.N + j) * kD);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float g0 = __uint_as_float(v[2 * e]) + s_bg[h * kD + 2 * e];
+            const float g1 = __uint_as_float(v[2 * e + 1]) + s_bg[h * kD + 2 * e + 1];
+            pk[e] = pack_bf16x2(__fdividef(1.0f, 1.0f + __expf(-g0)),
+                                __fdividef(1.0f, 1.0f + __expf(-g1)));
+          }
+          uint4* dst = reinterpret_cast<uint4*>(
+              a.G + (static_cast<long long>(r) * a.N + j) * kHD + h * kD);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+      tc_fence_before();
+      named_barrier_sync(bar_id, kGroupThreads);  // TMEM (and, after the second half, A) reused
+      tc_fence_after();
     }
-    const bool done = mbar_wait(mma_bar, mma_phase, abort_flag);
-    mma_phase ^= 1;
-    if (!__syncthreads_and(done ? 1 : 0)) {
-      if (tid == 0) report_status(a.status, kStatusTimeout);
+    if (!ok) {
+      if (gt == 0) report_status(a.status, kStatusTimeout);
       break;
     }
-    tc_fence_after();
-
-    // ---- epilogue: TMEM lane tid -> q, k, v, g of pair j
-#pragma unroll 1
-    for (int cc = 0; cc < 16; ++cc) {
-      uint32_t v[32];
-      tmem_ld32(tmem + lane_base + cc * 32, v);
-      tmem_ld_wait();
-      if (!jv) continue;
-      const int part = cc >> 2, h = cc & 3;
-      uint32_t pk[16];
-      if (part < 3) {
-        const float sc = part == 0 ? a.q_scale : 1.0f;
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
-        __nv_bfloat16* base = part == 0 ? a.Q : (part == 1 ? a.K : a.V);
-        uint4* dst = reinterpret_cast<uint4*>(
-            base + ((static_cast<long long>(r) * kHeads + h) * a.N + j) * kD);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float g0 = __uint_as_float(v[2 * e]) + s_bg[h * kD + 2 * e];
-          const float g1 = __uint_as_float(v[2 * e + 1]) + s_bg[h * kD + 2 * e + 1];
-          pk[e] = pack_bf16x2(__fdividef(1.0f, 1.0f + __expf(-g0)),
-                              __fdividef(1.0f, 1.0f + __expf(-g1)));
-        }
-        uint4* dst = reinterpret_cast<uint4*>(a.G + (static_cast<long long>(r) * a.N + j) * kHD +
-                                              h * kD);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-      }
-    }
-    tc_fence_before();
-    __syncthreads();  // A tile and TMEM are reused by the next tile
-    tc_fence_after();
   }
 
   // ---- teardown: never leave a bulk copy in flight into this CTA's smem
   if (tid == 0 && qkvg && !w_ready) {
-    if (!mbar_wait(w_bar, 0, nullptr))
-      report_status(a.status, kStatusTimeout);
+    if (!mbar_wait(w_bar, 0, nullptr)) report_status(a.status, kStatusTimeout);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0 && qkvg) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(*tmem_slot, kTmemCols);
   }
 }
 

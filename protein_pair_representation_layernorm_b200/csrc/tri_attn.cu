@@ -434,7 +434,8 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
     a.ld_bias = ld;
     a.status = h->status;
     const long long ntiles = static_cast<long long>(nrows) * jtiles;
-    const unsigned grid = static_cast<unsigned>(std::min<long long>(ntiles, h->num_sms));
+    const unsigned grid = static_cast<unsigned>(
+        std::min<long long>((ntiles + tri::plp::kGroupsPerCta - 1) / tri::plp::kGroupsPerCta, h->num_sms));
     Timer tm(h, st, timed, 0);
     tri::plp::pair_ln_proj<<<grid, tri::plp::kThreads, tri::plp::kSmemBytes, st>>>(a);
     return cudaGetLastError();
