@@ -145,6 +145,35 @@ size_t tri_attn_workspace_bytes(tri_attn_dtype dtype, int N);
 int tri_attn_debug_workspace(tri_attn_handle *h, void **q, void **k, void **v, void **g,
                              void **bias, void **o, int *ld_bias, int *rows);
 
+/* One forward of the bf16 block that allocates no device memory at all.
+ *
+ * For callers that are not allowed to call cudaMalloc: code embedded in a host
+ * application that owns every byte of device memory through its own pool or
+ * budget, and latency-critical paths where the implicit synchronisation and
+ * unpredictable cost of a device allocation is not acceptable.  Such callers
+ * cannot create a handle (tri_attn_create allocates), so this entry point takes
+ * the weights directly (`params`, device pointers, bf16 only) together with the
+ * usual Z, mask, out, N, orientation and stream; the arguments mean what they
+ * mean for tri_attn_forward.  There is no counterpart of this call on the pages
+ * this library follows.
+ *
+ * Scratch: everything besides the caller's buffers (the repacked weights, the
+ * status word and the workspace) lives in one statically allocated device array
+ * of 32 MiB inside this library; every GPU that loads the library holds it
+ * until the process exits.  Rows are processed in chunks that fit the array.
+ * Sizes it cannot hold (the whole logit bias plus one four-row chunk must fit,
+ * which allows N up to about 1750) return TRI_ATTN_ERR_UNSUPPORTED before
+ * anything is launched.  The first call on a device also looks up the array's
+ * device address (cudaGetSymbolAddress); make that first call before any stream
+ * capture.  All calls share the one array, which keeps the last call's contents
+ * (the status word is cleared at the start of each call): calls that overlap on
+ * the GPU, e.g. on two streams of the same device, race and corrupt each other;
+ * serialise them.  Flags: TRI_ATTN_FLAG_SYNC synchronises the stream and returns
+ * the device status; the other flags are ignored. */
+int tri_attn_forward_noalloc(const tri_attn_params *params, const void *Z, int N,
+                             const uint8_t *mask, tri_attn_orientation orientation, void *out,
+                             void *stream, unsigned flags);
+
 /* Release everything the handle owns.  NULL-safe.  Not stream-ordered:
  * call it after the work that uses the handle has completed. */
 int tri_attn_destroy(tri_attn_handle *h);

@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.tri_attn_workspace_bytes.restype = sz
         L.tri_attn_debug_workspace.argtypes = [vp] + [ctypes.POINTER(vp)] * 6 + [
             ctypes.POINTER(ci), ctypes.POINTER(ci)]
+        L.tri_attn_forward_noalloc.argtypes = [ctypes.POINTER(tri_attn_params), vp, ci, vp, ci,
+                                               vp, vp, cu]
         L.tri_attn_destroy.argtypes = [vp]
         L.tri_attn_status_string.argtypes = [ci]
         L.tri_attn_status_string.restype = ctypes.c_char_p
@@ -159,6 +161,13 @@ def tri_attn_debug_workspace(h) -> dict:
     d["ld_bias"] = ld.value
     d["rows"] = rows.value
     return d
+
+
+def tri_attn_forward_noalloc(params: tri_attn_params, Z_ptr, N: int, mask_ptr, orientation: int,
+                             out_ptr, stream=None, flags: int = 0) -> int:
+    """Forward that allocates no device memory (bf16 only); see tri_attn.h."""
+    return lib().tri_attn_forward_noalloc(ctypes.byref(params), Z_ptr, int(N), mask_ptr,
+                                          int(orientation), out_ptr, stream, int(flags))
 
 
 def tri_attn_destroy(h) -> int:

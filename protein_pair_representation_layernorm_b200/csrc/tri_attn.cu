@@ -20,6 +20,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -744,3 +745,162 @@ int tri_attn_destroy(tri_attn_handle* h) {
 }
 
 }  // extern "C"
+
+// ===================================================================== no-alloc
+// Entry point for callers that cannot allocate device memory (see
+// tri_attn_forward_noalloc in tri_attn.h).  Everything the block needs beyond the
+// caller's own buffers lives in one file-scope device array: the packed weight
+// images, the fp32 parameters, the device status word and the workspace.  The
+// existing kernels run on it unchanged, in row chunks sized to the array.
+namespace {
+
+constexpr size_t kNoallocScratchBytes = size_t(32) << 20;  // 32 MiB per device
+constexpr size_t kNaWImg = 0;                                // 512 x 128 bf16 image
+constexpr size_t kNaWoImg = kNaWImg + 512 * 128 * 2;         // 128 x 128 bf16 image
+constexpr size_t kNaWb = kNaWoImg + 128 * 128 * 2;           // fp32 [H][c_z] x log2(e)
+constexpr size_t kNaGamma = kNaWb + kHeads * kCz * 4;
+constexpr size_t kNaBeta = kNaGamma + kCz * 4;
+constexpr size_t kNaBg = kNaBeta + kCz * 4;
+constexpr size_t kNaBo = kNaBg + kHD * 4;
+constexpr size_t kNaStatus = kNaBo + kCz * 4;
+constexpr size_t kNaWs = (kNaStatus + 256 + 1023) / 1024 * 1024;  // workspace: the rest
+constexpr int kNaMaxDevices = 64;
+
+// Device memory of the library itself: present on every GPU that loads it,
+// until the process exits.  In host code this name is only a stand-in; the
+// device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kNaMaxDevices] = {};
+
+// Byte offset of element (n, k) in the K-major, 128-byte-swizzled image of a
+// bf16 operand with `rows` rows of 128 elements (same layout as
+// pack_kmajor_sw128 above).
+__device__ __forceinline__ size_t sw128_offset(int rows, int n, int k) {
+  const int slab = k / 64, c = (k % 64) / 8, e = k % 8;
+  return static_cast<size_t>(slab) * rows * 128 + static_cast<size_t>(n) * 128 +
+         ((c ^ (n & 7)) * 16) + e * 2;
+}
+
+// Repack the caller's bf16 weights into the scratch array, on the stream.
+__global__ void pack_weights_noalloc(const bf16* wq, const bf16* wk, const bf16* wv,
+                                     const bf16* wg, const bf16* wo, const bf16* wb,
+                                     const bf16* gamma, const bf16* beta, const bf16* bg,
+                                     const bf16* bo, unsigned char* scratch) {
+  const int n_w = 512 * 128, n_wo = 128 * 128, n_wb = kHeads * kCz;
+  const int total = n_w + n_wo + n_wb + 4 * kCz;
+  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += gridDim.x * blockDim.x) {
+    if (idx < n_w) {
+      const int n = idx / 128, k = idx % 128, part = n / kHD, nn = n % kHD;
+      const bf16* src = part == 0 ? wq : part == 1 ? wk : part == 2 ? wv : wg;
+      *reinterpret_cast<bf16*>(scratch + kNaWImg + sw128_offset(512, n, k)) = src[nn * kCz + k];
+    } else if (idx < n_w + n_wo) {
+      const int t = idx - n_w, n = t / 128, k = t % 128;
+      *reinterpret_cast<bf16*>(scratch + kNaWoImg + sw128_offset(128, n, k)) = wo[n * kHD + k];
+    } else if (idx < n_w + n_wo + n_wb) {
+      const int t = idx - n_w - n_wo;
+      reinterpret_cast<float*>(scratch + kNaWb)[t] = __bfloat162float(wb[t]) * tri::kLog2e;
+    } else {
+      const int t = idx - n_w - n_wo - n_wb, which = t / kCz, c = t % kCz;
+      if (which == 0) reinterpret_cast<float*>(scratch + kNaGamma)[c] = __bfloat162float(gamma[c]);
+      if (which == 1) reinterpret_cast<float*>(scratch + kNaBeta)[c] = __bfloat162float(beta[c]);
+      if (which == 2)
+        reinterpret_cast<float*>(scratch + kNaBg)[c] = bg ? __bfloat162float(bg[c]) : 0.f;
+      if (which == 3)
+        reinterpret_cast<float*>(scratch + kNaBo)[c] = bo ? __bfloat162float(bo[c]) : 0.f;
+    }
+  }
+}
+
+// Scratch a forward of size N needs: the weights, the whole bias and at least one
+// chunk of rows (the attention kernel's row group).
+size_t noalloc_required(int N) {
+  return kNaWs + bias_bytes(TRI_ATTN_BF16, N) + 6 * 256 +
+         static_cast<size_t>(tri::attn::kRows) * row_bytes(TRI_ATTN_BF16, N);
+}
+
+}  // namespace
+
+extern "C" int tri_attn_forward_noalloc(const tri_attn_params* p, const void* Z, int N,
+                                        const uint8_t* mask, tri_attn_orientation orientation,
+                                        void* out, void* stream, unsigned flags) {
+  if (!p || !Z || !out || N < 1) return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->dtype != TRI_ATTN_BF16) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (p->c_z != kCz || p->n_heads != kHeads || p->head_dim != kD) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (!p->ln_gamma || !p->ln_beta || !p->w_q || !p->w_k || !p->w_v || !p->w_g || !p->w_b ||
+      !p->w_o)
+    return TRI_ATTN_ERR_INVALID_ARG;
+  if (!(p->ln_eps >= 0.f) || !std::isfinite(p->ln_eps)) return TRI_ATTN_ERR_INVALID_ARG;
+  if (orientation != TRI_ATTN_STARTING && orientation != TRI_ATTN_ENDING)
+    return TRI_ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(Z) & 15) || (reinterpret_cast<uintptr_t>(out) & 15))
+    return TRI_ATTN_ERR_INVALID_ARG;
+  if (N > 46340 || noalloc_required(N) > kNoallocScratchBytes) {
+    TA_LOG("tri_attn_forward_noalloc: N=%d needs %zu bytes of scratch, the static array holds %zu",
+           N, noalloc_required(N), kNoallocScratchBytes);
+    return TRI_ATTN_ERR_UNSUPPORTED;
+  }
+  const size_t bytes = static_cast<size_t>(N) * N * kCz * 2;
+  if (Z != out && ranges_overlap(Z, out, bytes)) return TRI_ATTN_ERR_ALIAS;
+  int rc = check_device();
+  if (rc != TRI_ATTN_OK) return rc;
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kNaMaxDevices) return TRI_ATTN_ERR_UNSUPPORTED;
+
+  // set-up, once per device, with that device current
+  void* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_addr[dev]) {
+      void* ptr = nullptr;
+      CUDA_TRY(cudaGetSymbolAddress(&ptr, g_noalloc_scratch));
+      g_noalloc_addr[dev] = ptr;
+    }
+    base = g_noalloc_addr[dev];
+  }
+  unsigned char* scratch = static_cast<unsigned char*>(base);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // the array keeps the previous call's contents: the status word must start at 0
+  CUDA_TRY(cudaMemsetAsync(scratch + kNaStatus, 0, sizeof(int), st));
+  pack_weights_noalloc<<<128, 256, 0, st>>>(
+      static_cast<const bf16*>(p->w_q), static_cast<const bf16*>(p->w_k),
+      static_cast<const bf16*>(p->w_v), static_cast<const bf16*>(p->w_g),
+      static_cast<const bf16*>(p->w_o), static_cast<const bf16*>(p->w_b),
+      static_cast<const bf16*>(p->ln_gamma), static_cast<const bf16*>(p->ln_beta),
+      static_cast<const bf16*>(p->b_g), static_cast<const bf16*>(p->b_o), scratch);
+  CUDA_TRY(cudaGetLastError());
+
+  // a handle on the stack whose buffers all point into the scratch array, so the
+  // forward below never reaches cudaMalloc
+  tri_attn_handle hh;
+  hh.device = dev;
+  cudaDeviceGetAttribute(&hh.num_sms, cudaDevAttrMultiProcessorCount, dev);
+  hh.dtype = TRI_ATTN_BF16;
+  hh.eps = p->ln_eps;
+  hh.q_scale = tri::kLog2e / std::sqrt(static_cast<float>(kD));
+  hh.w_qkvg = scratch + kNaWImg;
+  hh.w_o = scratch + kNaWoImg;
+  hh.w_b = reinterpret_cast<float*>(scratch + kNaWb);
+  hh.gamma = reinterpret_cast<float*>(scratch + kNaGamma);
+  hh.beta = reinterpret_cast<float*>(scratch + kNaBeta);
+  hh.b_g = reinterpret_cast<float*>(scratch + kNaBg);
+  hh.b_o = reinterpret_cast<float*>(scratch + kNaBo);
+  hh.status = reinterpret_cast<int*>(scratch + kNaStatus);
+  hh.ws = scratch + kNaWs;
+  hh.ws_bytes = kNoallocScratchBytes - kNaWs;
+  hh.ws_limit = hh.ws_bytes;
+  rc = forward_impl(&hh, Z, N, mask, static_cast<int>(orientation), out, st,
+                    flags & ~(TRI_ATTN_FLAG_TIME_KERNELS | TRI_ATTN_FLAG_DEBUG_STALL));
+  if (rc == TRI_ATTN_OK && (flags & TRI_ATTN_FLAG_SYNC)) {
+    int s = 0;
+    CUDA_TRY(cudaMemcpyAsync(&s, hh.status, sizeof(int), cudaMemcpyDeviceToHost, st));
+    CUDA_TRY(cudaStreamSynchronize(st));
+    rc = s;
+  }
+  hh.ws = nullptr;  // nothing in hh is owned: the handle is never destroyed
+  return rc;
+}
