@@ -1,16 +1,19 @@
 // gate_out.cuh — sigmoid gate, output projection (tcgen05) and residual add,
 // bf16 pair representation.
 //
-// One CTA of 128 threads handles 128 pairs (i, j0..j0+127) of one problem row.
-// Thread t owns pair j0+t: it forms  g * o  (g = sigmoid gate already applied
-// by pair_ln_proj, o = attention output of the 4 heads), rounds it to bf16 and
-// writes it into the MMA A tile (K-major, 128-byte swizzle).  Thread 0 issues 8
-// tcgen05 MMAs, D[128 x 128] = (G*O) Wo^T, fp32 in 128 TMEM columns; each
-// thread then adds bo and its own residual z_ij (loaded at the start, together
-// with o and g, so that all of a thread's loads are in flight at once) and writes
-// out_ij as bf16 with 16-byte vector stores.  The ending-node block reads the residual from and
-// writes the result to the swapped view (pair (i, j) is Z[j][i]).  A thread
-// reads z_ij before writing out_ij, so out may alias Z.
+// Persistent CTAs walk tiles of 128 pairs (i, j0..j0+127) of one problem row
+// through a two-stage pipeline.  A producer warp moves each tile in with TMA:
+// o (4 head boxes of [128 pairs][32], 64-byte swizzle), g ([128][128], 128-byte
+// swizzle) and the residual z ([128][128], 128-byte swizzle; the ending-node
+// block reads the swapped view, pair (i, j) = Z[j][i], as a box that is one
+// pair wide and 128 pairs deep).  Thread t of the four compute warps owns pair
+// j0+t: it forms bf16(g * o) in place over g, which already has the layout of
+// the MMA A operand (K-major, 128-byte swizzle); one thread issues 8 tcgen05
+// MMAs, D[128 x 128] = (G*O) Wo^T with Wo resident in shared memory, into one of
+// two 128-column TMEM accumulators; each thread then adds bo and z and writes
+// out_ij in place over z, and one thread stores the tile with TMA (through the
+// swapped view again for the ending node).  Every element of out is read (as z)
+// and written by the same CTA, tile by tile, so out may alias Z.
 //
 // HBM-bound: per pair it reads 768 B (o, g, z) and writes 256 B.
 #pragma once
@@ -21,36 +24,68 @@
 namespace tri {
 namespace gout {
 
-constexpr int kThreads = 128;
+constexpr int kComputeThreads = 128;
+constexpr int kThreads = kComputeThreads + 32;   // + producer warp
+constexpr int kProducerWarp = 4;
 constexpr int kTileM = 128;
+constexpr int kStages = 2;
 constexpr uint32_t kWoBytes = kCz * kHD * 2;     // 32768
 constexpr uint32_t kWoAtomBytes = kCz * 128;     // 16384
-constexpr uint32_t kATileBytes = kTileM * kHD * 2;
-constexpr uint32_t kAAtomBytes = kTileM * 128;
+constexpr uint32_t kOHeadBytes = kTileM * kD * 2;    // 8192: [128 pairs][32] bf16
+constexpr uint32_t kSlabBytes = kTileM * 128;        // 16384: [128 pairs][64] bf16
+constexpr uint32_t kStO = 0;
+constexpr uint32_t kStG = kHeads * kOHeadBytes;      // 32768
+constexpr uint32_t kStZ = kStG + 2 * kSlabBytes;     // 65536
+constexpr uint32_t kStageBytes = kStZ + 2 * kSlabBytes;  // 98304
 constexpr uint32_t kSmemW = 0;
-constexpr uint32_t kSmemA = kWoBytes;
-constexpr uint32_t kSmemBo = kSmemA + kATileBytes;
+constexpr uint32_t kSmemStages = kWoBytes;
+constexpr uint32_t kSmemBo = kSmemStages + kStages * kStageBytes;
 constexpr uint32_t kSmemBar = kSmemBo + kCz * 4;
-constexpr uint32_t kSmemBytes = kSmemBar + 64 + 1024;
-constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kNumBars = 1 + 3 * kStages;
+constexpr uint32_t kSmemBytes = kSmemBar + kNumBars * 8 + 16 + 1024;
+constexpr uint32_t kTmemCols = 256;  // two 128-column accumulators
 
-__global__ void __launch_bounds__(kThreads) gate_out(const GateArgs a) {
+// TMA store of a box from shared memory (bulk-group completion).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0,
+                                             int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gate_out(const __grid_constant__ CUtensorMap map_o, const __grid_constant__ CUtensorMap map_g,
+             const __grid_constant__ CUtensorMap map_z, const __grid_constant__ CUtensorMap map_out,
+             const GateArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sW = smem + kSmemW;
-  uint8_t* sA = smem + kSmemA;
   float* s_bo = reinterpret_cast<float*>(smem + kSmemBo);
-  uint64_t* w_bar = reinterpret_cast<uint64_t*>(smem + kSmemBar);
-  uint64_t* mma_bar = w_bar + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(w_bar + 2);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemBar);
+  uint64_t* w_bar = bars;
+  uint64_t* full = bars + 1;
+  uint64_t* empty = full + kStages;
+  uint64_t* mma_bar = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int idx = tid; idx < kCz; idx += kThreads) s_bo[idx] = a.b_o[idx];
   if (tid == 0) {
     mbar_init(w_bar, 1);
-    mbar_init(mma_bar, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&mma_bar[s], 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -62,113 +97,175 @@ __global__ void __launch_bounds__(kThreads) gate_out(const GateArgs a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (tid == 0) {
-    mbar_arrive_expect_tx(w_bar, kWoBytes);
-    bulk_load(sW, a.wo_img, kWoBytes, w_bar);
-  }
 
-  const int r = blockIdx.y;
-  const int i = a.row0 + r;
-  const int j = blockIdx.x * kTileM + tid;
-  const bool jv = j < a.N;
-
-  // ---- the residual pair vector: loaded now so that it is in flight with o and g
-  const long long zoff = jv ? pair_offset(a.orient, a.N, i, j) : 0;
-  uint4 zv[16];
-  if (jv) {
-    const uint4* zp = reinterpret_cast<const uint4*>(a.Z + zoff);
-#pragma unroll
-    for (int q = 0; q < 16; ++q) zv[q] = zp[q];
-  }
-
-  // ---- A = bf16(g * o), K index = h*d + e
-#pragma unroll
-  for (int h = 0; h < kHeads; ++h) {
-    uint4 ov[4], gv[4];
-    if (jv) {
-      const uint4* op = reinterpret_cast<const uint4*>(
-          a.O + ((static_cast<long long>(r) * kHeads + h) * a.N + j) * kD);
-      const uint4* gp = reinterpret_cast<const uint4*>(
-          a.G + (static_cast<long long>(r) * a.N + j) * kHD + h * kD);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        ov[q] = __ldg(op + q);
-        gv[q] = __ldg(gp + q);
-      }
+  const int jtiles = (a.N + kTileM - 1) / kTileM;
+  const long long ntiles = static_cast<long long>(a.rows) * jtiles;
+  // TMA coordinates of the z / out box of a tile: (channel, column, row) of Z
+  auto zcoords = [&](long long tile, int& c1, int& c2) {
+    const int r = static_cast<int>(tile / jtiles);
+    const int j0 = static_cast<int>(tile % jtiles) * kTileM;
+    const int i = a.row0 + r;
+    if (a.orient == 0) {
+      c1 = j0;
+      c2 = i;
     } else {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) ov[q] = gv[q] = make_uint4(0, 0, 0, 0);
+      c1 = i;
+      c2 = j0;
     }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t ow[4] = {ov[q].x, ov[q].y, ov[q].z, ov[q].w};
-      const uint32_t gw[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
-      uint32_t pk[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        pk[e] = pack_bf16x2(bf16lo_to_f32(ow[e]) * bf16lo_to_f32(gw[e]),
-                            bf16hi_to_f32(ow[e]) * bf16hi_to_f32(gw[e]));
-      const int c = h * 4 + q;  // 16-byte chunk along K
-      uint8_t* dst = sA + (c >> 3) * kAAtomBytes + tid * 128 + (((c & 7) ^ (tid & 7)) << 4);
-      *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    }
-  }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
+  };
 
-  if (tid == 0) {
-    if (mbar_wait(w_bar, 0, abort_flag)) {
-      constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, false);
-      const uint32_t sA_u32 = smem_u32(sA), sW_u32 = smem_u32(sW);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t ad =
-            smem_desc(sA_u32 + (kk >> 2) * kAAtomBytes + (kk & 3) * 32, 1024, kSwizzle128B);
-        const uint64_t bd =
-            smem_desc(sW_u32 + (kk >> 2) * kWoAtomBytes + (kk & 3) * 32, 1024, kSwizzle128B);
-        mma_ss(tmem, ad, bd, kIdesc, kk > 0 ? 1u : 0u);
-      }
-      mma_commit(mma_bar);
-    } else {
-      *abort_flag = 1;
-      report_status(a.status, kStatusTimeout);
-      mbar_wait(w_bar, 0, nullptr);  // do not exit with the copy in flight
-    }
-  }
-  const bool done = mbar_wait(mma_bar, 0, abort_flag);
-  if (__syncthreads_and(done ? 1 : 0)) {
-    tc_fence_after();
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      uint32_t v[32];
-      tmem_ld32(tmem + lane_base + cc * 32, v);
-      tmem_ld_wait();
-      if (!jv) continue;
-      uint32_t pk[16];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 zq = zv[cc * 4 + q];
-        const uint32_t zw[4] = {zq.x, zq.y, zq.z, zq.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c0 = cc * 32 + q * 8 + 2 * e;
-          const float y0 = __uint_as_float(v[q * 8 + 2 * e]) + s_bo[c0] + bf16lo_to_f32(zw[e]);
-          const float y1 =
-              __uint_as_float(v[q * 8 + 2 * e + 1]) + s_bo[c0 + 1] + bf16hi_to_f32(zw[e]);
-          pk[q * 4 + e] = pack_bf16x2(y0, y1);
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&map_o);
+      tma_prefetch_desc(&map_g);
+      tma_prefetch_desc(&map_z);
+      mbar_arrive_expect_tx(w_bar, kWoBytes);
+      bulk_load(smem + kSmemW, a.wo_img, kWoBytes, w_bar);
+      long long n_issued = 0;
+      for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++n_issued) {
+        const int s = static_cast<int>(n_issued % kStages);
+        if (n_issued >= kStages &&
+            !mbar_wait(&empty[s], static_cast<uint32_t>((n_issued / kStages) - 1) & 1,
+                       abort_flag)) {
+          *abort_flag = 1;
+          report_status(a.status, kStatusTimeout);
+          break;
+        }
+        uint8_t* st = smem + kSmemStages + s * kStageBytes;
+        const int r = static_cast<int>(tile / jtiles);
+        const int j0 = static_cast<int>(tile % jtiles) * kTileM;
+        int c1, c2;
+        zcoords(tile, c1, c2);
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        for (int h = 0; h < kHeads; ++h)
+          tma_load_3d(st + kStO + h * kOHeadBytes, &map_o, &full[s], 0, j0, r * kHeads + h);
+        for (int slab = 0; slab < 2; ++slab) {
+          tma_load_3d(st + kStG + slab * kSlabBytes, &map_g, &full[s], 64 * slab, j0, r);
+          tma_load_3d(st + kStZ + slab * kSlabBytes, &map_z, &full[s], 64 * slab, c1, c2);
         }
       }
-      uint4* op = reinterpret_cast<uint4*>(a.out + zoff + cc * 32);
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        op[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      // never leave a copy in flight into this CTA's shared memory
+      if (!mbar_wait(w_bar, 0, nullptr)) report_status(a.status, kStatusTimeout);
+      for (long long n = n_issued - kStages; n < n_issued; ++n)
+        if (n >= 0 &&
+            !mbar_wait(&full[n % kStages], static_cast<uint32_t>(n / kStages) & 1, nullptr))
+          report_status(a.status, kStatusTimeout);
     }
-  } else if (tid == 0) {
-    report_status(a.status, kStatusTimeout);
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ compute
+    const int gt = tid;                     // pair within the tile = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t sW_u32 = smem_u32(smem + kSmemW);
+    constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, false);
+    bool w_ready = false, ok = true, stored = false;
+    long long n = 0;
+    for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++n) {
+      const int s = static_cast<int>(n % kStages);
+      const uint32_t ph = static_cast<uint32_t>(n / kStages) & 1;
+      uint8_t* st = smem + kSmemStages + s * kStageBytes;
+      if (!named_barrier_and(1, kComputeThreads, mbar_wait(&full[s], ph, abort_flag))) {
+        ok = false;
+        break;
+      }
+      // ---- A = bf16(g * o) in place over g (16-byte chunk c = channels 8c..8c+7)
+      uint8_t* grow = st + kStG + gt * 128;
+      const uint8_t* orow = st + kStO + gt * 64;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const int h = c >> 2, q = c & 3;
+        uint8_t* gp = grow + (c >> 3) * kSlabBytes + (((c & 7) ^ (gt & 7)) << 4);
+        const uint4 gv = *reinterpret_cast<const uint4*>(gp);
+        const uint4 ov = *reinterpret_cast<const uint4*>(orow + h * kOHeadBytes +
+                                                         ((q ^ ((gt >> 1) & 3)) << 4));
+        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+        const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          pk[e] = pack_bf16x2(bf16lo_to_f32(ow[e]) * bf16lo_to_f32(gw[e]),
+                              bf16hi_to_f32(ow[e]) * bf16hi_to_f32(gw[e]));
+        *reinterpret_cast<uint4*>(gp) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_barrier_sync(1, kComputeThreads);
+      tc_fence_after();
+      const uint32_t acc = tmem + s * 128;
+      if (gt == 0) {
+        bool ready = true;
+        if (!w_ready) ready = w_ready = mbar_wait(w_bar, 0, abort_flag);
+        if (ready) {
+          const uint32_t sA = smem_u32(st + kStG);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t ad = smem_desc(sA + (kk >> 2) * kSlabBytes + (kk & 3) * 32, 1024,
+                                          kSwizzle128B);
+            const uint64_t bd = smem_desc(sW_u32 + (kk >> 2) * kWoAtomBytes + (kk & 3) * 32,
+                                          1024, kSwizzle128B);
+            mma_ss(acc, ad, bd, kIdesc, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&mma_bar[s]);
+        } else {
+          *abort_flag = 1;
+          report_status(a.status, kStatusTimeout);
+        }
+      }
+      if (!named_barrier_and(1, kComputeThreads, mbar_wait(&mma_bar[s], ph, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // ---- out = acc + bo + z, in place over z
+      uint8_t* zrow = st + kStZ + gt * 128;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(acc + lane_base + cc * 32, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c = cc * 4 + q;  // 16-byte chunk of the 128 channels
+          uint8_t* zp = zrow + (c >> 3) * kSlabBytes + (((c & 7) ^ (gt & 7)) << 4);
+          const uint4 zv = *reinterpret_cast<const uint4*>(zp);
+          const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int ch = c * 8 + 2 * e;
+            const float y0 = __uint_as_float(v[q * 8 + 2 * e]) + s_bo[ch] + bf16lo_to_f32(zw[e]);
+            const float y1 =
+                __uint_as_float(v[q * 8 + 2 * e + 1]) + s_bo[ch + 1] + bf16hi_to_f32(zw[e]);
+            pk[e] = pack_bf16x2(y0, y1);
+          }
+          *reinterpret_cast<uint4*>(zp) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_barrier_sync(1, kComputeThreads);
+      if (gt == 0) {
+        int c1, c2;
+        zcoords(tile, c1, c2);
+        for (int slab = 0; slab < 2; ++slab)
+          tma_store_3d(&map_out, st + kStZ + slab * kSlabBytes, 64 * slab, c1, c2);
+        bulk_commit();
+        stored = true;
+        bulk_wait_read_all();  // the stage's shared memory may be refilled after this
+        mbar_arrive(&empty[s]);
+      }
+    }
+    if (!ok && gt == 0) {
+      *abort_flag = 1;
+      report_status(a.status, kStatusTimeout);
+    }
+    if (gt == 0 && stored) {
+      // the stores must be complete (not only read out of shared memory) at exit
+      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    }
   }
+
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

@@ -93,12 +93,13 @@ EncodeTiledFn encode_fn() {
 
 // 3-D bf16 tensor map; dims/strides innermost first, strides in bytes (dims 1, 2).
 bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-                 uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw) {
+                 uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw,
+                 uint32_t b2 = 1) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {d0, d1, d2};
   const cuuint64_t strides[2] = {s1, s2};
-  const cuuint32_t box[3] = {b0, b1, 1};
+  const cuuint32_t box[3] = {b0, b1, b2};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -472,6 +473,20 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
       CUDA_TRY(cudaGetLastError());
     }
     {
+      // o, g: this chunk's workspace; z, out: the pair tensor, boxes of 128 pairs
+      // along j (starting node) or, through the swapped view, along the rows of Z
+      CUtensorMap mo, mg, mz, mout;
+      const uint64_t rowb = static_cast<uint64_t>(N) * kCz * 2;
+      const uint32_t zb1 = orient == 0 ? 128u : 1u, zb2 = orient == 0 ? 1u : 128u;
+      bool okm =
+          make_map_3d(&mo, h->o, kD, N, static_cast<uint64_t>(nr) * kHeads, kD * 2,
+                      static_cast<uint64_t>(N) * kD * 2, kD, 128, CU_TENSOR_MAP_SWIZZLE_64B) &&
+          make_map_3d(&mg, h->g, kHD, N, nr, kHD * 2, static_cast<uint64_t>(N) * kHD * 2, 64, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B) &&
+          make_map_3d(&mz, Zb, kCz, N, N, kCz * 2, rowb, 64, zb1, CU_TENSOR_MAP_SWIZZLE_128B, zb2) &&
+          make_map_3d(&mout, outb, kCz, N, N, kCz * 2, rowb, 64, zb1, CU_TENSOR_MAP_SWIZZLE_128B,
+                      zb2);
+      if (!okm) return TRI_ATTN_ERR_CUDA;
       tri::GateArgs a{};
       a.Z = Zb;
       a.O = static_cast<const bf16*>(h->o);
@@ -484,9 +499,11 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
       a.row0 = r0;
       a.rows = nr;
       a.status = h->status;
-      dim3 grid(jtiles, nr);
+      const long long ntiles = static_cast<long long>(nr) * jtiles;
+      const unsigned grid = static_cast<unsigned>(std::min<long long>(ntiles, h->num_sms));
       Timer tm(h, st, timed, 2);
-      tri::gout::gate_out<<<grid, tri::gout::kThreads, tri::gout::kSmemBytes, st>>>(a);
+      tri::gout::gate_out<<<grid, tri::gout::kThreads, tri::gout::kSmemBytes, st>>>(mo, mg, mz,
+                                                                                   mout, a);
       CUDA_TRY(cudaGetLastError());
     }
   }
