@@ -136,7 +136,7 @@ size_t tri_attn_workspace_bytes(tri_attn_dtype dtype, int N);
 
 /* Device pointers of the intermediate tensors of the last forward call (for
  * inspection by tests).  Layouts, for rows r of the last chunk and head h:
- *   q, k, v, o: [rows][H][N][d];  g: [rows][N][H*d];  bias: [H][N][ld_bias]
+ *   q, k, v, g, o: [rows][H][N][d];  bias: [H][N][ld_bias]
  * (bias already scaled by log2(e); at masked keys and at columns >= N it is
  * -inf for F32 handles and -3e38 for BF16 handles, whose attention kernel adds
  * the bias with an MMA, where -inf would turn 0 * b into NaN;

@@ -3,12 +3,13 @@
 //
 // Persistent CTAs walk tiles of 128 pairs (i, j0..j0+127) of one problem row
 // through a two-stage pipeline.  A producer warp moves each tile in with TMA:
-// o (4 head boxes of [128 pairs][32], 64-byte swizzle), g ([128][128], 128-byte
-// swizzle) and the residual z ([128][128], 128-byte swizzle; the ending-node
-// block reads the swapped view, pair (i, j) = Z[j][i], as a box that is one
-// pair wide and 128 pairs deep).  Thread t of the four compute warps owns pair
-// j0+t: it forms bf16(g * o) in place over g, which already has the layout of
-// the MMA A operand (K-major, 128-byte swizzle); one thread issues 8 tcgen05
+// o and g (4 head boxes each of [128 pairs][32], 64-byte swizzle) and the
+// residual z ([128][128], 128-byte swizzle; the ending-node block reads the
+// swapped view, pair (i, j) = Z[j][i], as a box that is one pair wide and 128
+// pairs deep).  Thread t of the four compute warps owns pair j0+t: it forms
+// bf16(g * o) and, once every thread has read its g, writes it over the g
+// buffer in the layout of the MMA A operand (K-major, 128-byte swizzle); one
+// thread issues 8 tcgen05
 // MMAs, D[128 x 128] = (G*O) Wo^T with Wo resident in shared memory, into one of
 // two 128-column TMEM accumulators; each thread then adds bo and z and writes
 // out_ij in place over z, and one thread stores the tile with TMA (through the
@@ -140,10 +141,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&full[s], kStageBytes);
         for (int h = 0; h < kHeads; ++h)
           tma_load_3d(st + kStO + h * kOHeadBytes, &map_o, &full[s], 0, j0, r * kHeads + h);
-        for (int slab = 0; slab < 2; ++slab) {
-          tma_load_3d(st + kStG + slab * kSlabBytes, &map_g, &full[s], 64 * slab, j0, r);
+        for (int h = 0; h < kHeads; ++h)
+          tma_load_3d(st + kStG + h * kOHeadBytes, &map_g, &full[s], 0, j0, r * kHeads + h);
+        for (int slab = 0; slab < 2; ++slab)
           tma_load_3d(st + kStZ + slab * kSlabBytes, &map_z, &full[s], 64 * slab, c1, c2);
-        }
       }
       // never leave a copy in flight into this CTA's shared memory
       if (!mbar_wait(w_bar, 0, nullptr)) report_status(a.status, kStatusTimeout);
@@ -169,25 +170,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
         break;
       }
-      // ---- A = bf16(g * o) in place over g (16-byte chunk c = channels 8c..8c+7)
-      uint8_t* grow = st + kStG + gt * 128;
-      const uint8_t* orow = st + kStO + gt * 64;
+      // ---- A = bf16(g * o): 16-byte chunk c = channels 8c..8c+7 = head c/4, part c%4
+      uint32_t pk[64];
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         const int h = c >> 2, q = c & 3;
-        uint8_t* gp = grow + (c >> 3) * kSlabBytes + (((c & 7) ^ (gt & 7)) << 4);
-        const uint4 gv = *reinterpret_cast<const uint4*>(gp);
-        const uint4 ov = *reinterpret_cast<const uint4*>(orow + h * kOHeadBytes +
-                                                         ((q ^ ((gt >> 1) & 3)) << 4));
+        const uint32_t off = h * kOHeadBytes + gt * 64 + ((q ^ ((gt >> 1) & 3)) << 4);
+        const uint4 gv = *reinterpret_cast<const uint4*>(st + kStG + off);
+        const uint4 ov = *reinterpret_cast<const uint4*>(st + kStO + off);
         const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
         const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
-        uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          pk[e] = pack_bf16x2(bf16lo_to_f32(ow[e]) * bf16lo_to_f32(gw[e]),
-                              bf16hi_to_f32(ow[e]) * bf16hi_to_f32(gw[e]));
-        *reinterpret_cast<uint4*>(gp) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          pk[4 * c + e] = pack_bf16x2(bf16lo_to_f32(ow[e]) * bf16lo_to_f32(gw[e]),
+                                      bf16hi_to_f32(ow[e]) * bf16hi_to_f32(gw[e]));
       }
+      named_barrier_sync(1, kComputeThreads);  // every g has been read: reuse its buffer for A
+      uint8_t* grow = st + kStG + gt * 128;
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        *reinterpret_cast<uint4*>(grow + (c >> 3) * kSlabBytes + (((c & 7) ^ (gt & 7)) << 4)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       fence_proxy_async_smem();
       tc_fence_before();
       named_barrier_sync(1, kComputeThreads);

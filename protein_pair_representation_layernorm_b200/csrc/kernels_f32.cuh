@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(kProjThreads) ln_proj_kernel(ProjArgsF32 a) {
     if (part == 0) a.Q[qkv_idx] = acc * a.q_scale;
     else if (part == 1) a.K[qkv_idx] = acc;
     else if (part == 2) a.V[qkv_idx] = acc;
-    else a.G[(static_cast<long long>(r) * a.N + j) * kHD + ch] = 1.0f / (1.0f + expf(-(acc + a.b_g[ch])));
+    else a.G[qkv_idx] = 1.0f / (1.0f + expf(-(acc + a.b_g[ch])));
   }
 }
 
@@ -127,8 +127,8 @@ __global__ void __launch_bounds__(kProjThreads) gate_out_kernel(GateArgsF32 a) {
   float* go = gs[t];
   for (int ch = 0; ch < kHD; ++ch) {
     const int h = ch / kD, e = ch % kD;
-    const float o = a.O[((static_cast<long long>(r) * kHeads + h) * a.N + j) * kD + e];
-    go[ch] = o * a.G[(static_cast<long long>(r) * a.N + j) * kHD + ch];
+    const long long idx = ((static_cast<long long>(r) * kHeads + h) * a.N + j) * kD + e;
+    go[ch] = a.O[idx] * a.G[idx];
   }
   const long long off = pair_offset(a.orient, a.N, i, j);
   const float* z = a.Z + off;

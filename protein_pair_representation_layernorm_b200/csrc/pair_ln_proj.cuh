@@ -2,20 +2,25 @@
 // bias, bf16 pair representation.
 //
 // Persistent CTAs of two independent 128-thread groups.  Each group walks its
-// own tiles of 128 pairs of one problem row (pairs (i, j0..j0+127)); thread t of
-// the group owns pair j0+t:
-//   1. reads its 256-byte pair vector (the ending-node block reads Z[j][i]),
+// own tiles of 128 pairs of one problem row (pairs (i, j0..j0+127)).  The tile of
+// Z arrives by TMA straight into the group's MMA A buffer (K-major, 128-byte
+// swizzle: two boxes of 64 channels; the ending-node block reads the swapped
+// view, pair (i, j) = Z[j][i], as a box one pair wide and 128 pairs deep).
+// Thread t of the group owns pair j0+t:
+//   1. reads its 256-byte pair vector from the buffer,
 //   2. LayerNorm in fp32 (mean, biased variance, rsqrt),
 //   3. the per-head logit bias  Wb x  in fp32 (Wb pre-scaled by log2 e;
 //      kMaskedLogit at masked keys and at the padding columns j >= N),
-//   4. writes x as bf16 into the group's MMA A tile in shared memory (K-major,
-//      128-byte swizzle), then prefetches the pair vector of its next tile.
+//   4. writes x as bf16 back in place, which makes the buffer the A operand.
+// The next tile's TMA is issued as soon as the projection has consumed the
+// buffer, so it overlaps the last epilogue.
 // One thread of the group then issues the projection D = X W^T in two halves of
 // N = 256 (q|k, then v|g), W = [Wq; Wk; Wv; Wg] resident in shared memory for the
 // whole kernel, each half accumulating in fp32 in the group's 256 TMEM columns.
-// Each thread reads back its TMEM lane and writes q (scaled by log2(e)/sqrt(d)),
-// k, v head-major ([rows][H][N][d]) and sigmoid(g + bg) pair-major
-// ([rows][N][H*d]), bf16.  While one group runs its MMAs the other normalises or
+// Each thread reads back its TMEM lane; q (scaled by log2(e)/sqrt(d)), k, v and
+// sigmoid(g + bg) are written head-major ([rows][H][N][d], bf16), each warp
+// staging its 32 pairs' 64-byte rows in shared memory so that the global stores
+// are contiguous 512-byte blocks.  While one group runs its MMAs the other normalises or
 // stores, so the tensor core, the ALUs and HBM overlap.
 //
 // This is the HBM-bound step: per pair it reads 256 B and writes 1 KB + 8 B.
@@ -40,26 +45,15 @@ constexpr uint32_t kSmemW = 0;
 constexpr uint32_t kSmemA = kWImgBytes;                                  // + grp * kATileBytes
 constexpr uint32_t kSmemPar = kSmemA + kGroupsPerCta * kATileBytes;     // fp32 params
 constexpr uint32_t kParFloats = kHeads * kCz + 3 * kCz;                 // w_b, gamma, beta, b_g
-constexpr uint32_t kSmemBar = kSmemPar + kParFloats * 4;
+constexpr uint32_t kSmemStg = kSmemPar + kParFloats * 4;               // per-warp store staging
+constexpr uint32_t kStgBytes = 32 * 64;                                 // 32 pairs x 64 B
+constexpr uint32_t kSmemBar = kSmemStg + (kThreads / 32) * kStgBytes;
 constexpr uint32_t kSmemBytes = kSmemBar + 64 + 1024;                   // + alignment slack
+static_assert(kGroupsPerCta * 2 * 8 + 8 + 8 <= 64, "barrier area");
 constexpr uint32_t kTmemCols = 512;                                     // 256 per group
 
-__device__ __forceinline__ void load_pair(const ProjArgs& a, long long tile, int jtiles, int gt,
-                                          uint4 (&zr)[16]) {
-  const int r = static_cast<int>(tile / jtiles);
-  const int j = static_cast<int>(tile % jtiles) * kTileM + gt;
-  if (j < a.N) {
-    const uint4* zp =
-        reinterpret_cast<const uint4*>(a.Z + pair_offset(a.orient, a.N, a.row0 + r, j));
-#pragma unroll
-    for (int c = 0; c < 16; ++c) zr[c] = __ldg(zp + c);
-  } else {
-#pragma unroll
-    for (int c = 0; c < 16; ++c) zr[c] = make_uint4(0, 0, 0, 0);
-  }
-}
-
-__global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
+__global__ void __launch_bounds__(kThreads, 1)
+    pair_ln_proj(const __grid_constant__ CUtensorMap map_z, const ProjArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -68,8 +62,9 @@ __global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
   float* s_beta = s_gamma + kCz;
   float* s_bg = s_beta + kCz;
   uint64_t* w_bar = reinterpret_cast<uint64_t*>(smem + kSmemBar);
-  uint64_t* mma_bar = w_bar + 1;  // one per group
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + kGroupsPerCta);
+  uint64_t* mma_bar = w_bar + 1;                // one per group
+  uint64_t* z_full = mma_bar + kGroupsPerCta;   // one per group
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(z_full + kGroupsPerCta);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -87,7 +82,10 @@ __global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
   }
   if (tid == 0) {
     mbar_init(w_bar, 1);
-    for (int g = 0; g < kGroupsPerCta; ++g) mbar_init(&mma_bar[g], 1);
+    for (int g = 0; g < kGroupsPerCta; ++g) {
+      mbar_init(&mma_bar[g], 1);
+      mbar_init(&z_full[g], 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -116,13 +114,37 @@ __global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
   const bool mma_thread = gt == 0;
 
   long long tile = static_cast<long long>(blockIdx.x) * kGroupsPerCta + grp;
-  uint4 zr[16];
-  if (tile < ntiles) load_pair(a, tile, jtiles, gt, zr);
+  // TMA of a tile of Z into this group's A buffer
+  auto issue_z = [&](long long t) {
+    const int r = static_cast<int>(t / jtiles);
+    const int j0 = static_cast<int>(t % jtiles) * kTileM;
+    const int i = a.row0 + r;
+    const int c1 = a.orient == 0 ? j0 : i, c2 = a.orient == 0 ? i : j0;
+    mbar_arrive_expect_tx(&z_full[grp], kATileBytes);
+    tma_load_3d(sA, &map_z, &z_full[grp], 0, c1, c2);
+    tma_load_3d(sA + kAAtomBytes, &map_z, &z_full[grp], 64, c1, c2);
+  };
+  if (mma_thread) tma_prefetch_desc(&map_z);
+  if (mma_thread && tile < ntiles) issue_z(tile);
+  uint32_t z_phase = 0;
+  bool z_pending = tile < ntiles;
   for (; tile < ntiles; tile += stride) {
     const int r = static_cast<int>(tile / jtiles);
     const int i = a.row0 + r;
     const int j = static_cast<int>(tile % jtiles) * kTileM + gt;
     const bool jv = j < a.N;
+
+    if (!named_barrier_and(bar_id, kGroupThreads, mbar_wait(&z_full[grp], z_phase, abort_flag))) {
+      if (gt == 0) report_status(a.status, kStatusTimeout);
+      break;
+    }
+    z_phase ^= 1;
+    z_pending = false;
+    uint4 zr[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+      zr[c] = *reinterpret_cast<const uint4*>(sA + (c >> 3) * kAAtomBytes + gt * 128 +
+                                              (((c & 7) ^ (gt & 7)) << 4));
 
     // ---- LayerNorm statistics in fp32 (two passes over registers)
     float sum = 0.f;
@@ -179,9 +201,15 @@ __global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
               __float2bfloat16_rn(key_valid ? bacc[h] : kMaskedLogit);
       }
     }
-    // ---- prefetch the next tile's pair vector while this one is projected
-    if (tile + stride < ntiles) load_pair(a, tile + stride, jtiles, gt, zr);
-    if (!qkvg) continue;
+    if (!qkvg) {
+      // bias only: the buffer is free once every thread of the group has read it
+      named_barrier_sync(bar_id, kGroupThreads);
+      if (mma_thread && tile + stride < ntiles) {
+        issue_z(tile + stride);
+        z_pending = true;
+      }
+      continue;
+    }
 
     fence_proxy_async_smem();
     tc_fence_before();
@@ -221,14 +249,22 @@ __global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
         break;
       }
       tc_fence_after();
+      if (half == 1 && mma_thread && tile + stride < ntiles) {
+        issue_z(tile + stride);  // the A buffer has been consumed by both MMAs
+        z_pending = true;
+      }
 
-      // ---- epilogue: TMEM lane gt -> two of q, k, v, g of pair j
+      // ---- epilogue: TMEM lane gt -> two of q, k, v, g of pair j.  Each 32-column
+      // chunk (one head of one output) of the warp's 32 pairs is 32 rows of 64 B,
+      // contiguous in the head-major output: the warp stages it in shared memory
+      // and writes it back with 512-byte coalesced stores.
+      const int jw0 = static_cast<int>(tile % jtiles) * kTileM + (warp & 3) * 32;
+      uint8_t* stg = smem + kSmemStg + warp * kStgBytes;
 #pragma unroll 1
       for (int cc = 0; cc < 8; ++cc) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_base + cc * 32, v);
         tmem_ld_wait();
-        if (!jv) continue;
         const int part = half * 2 + (cc >> 2), h = cc & 3;
         uint32_t pk[16];
         if (part < 3) {
@@ -236,12 +272,6 @@ __global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
-          __nv_bfloat16* base = part == 0 ? a.Q : (part == 1 ? a.K : a.V);
-          uint4* dst = reinterpret_cast<uint4*>(
-              base + ((static_cast<long long>(r) * kHeads + h) * a.N + j) * kD);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
         } else {
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -250,12 +280,25 @@ __global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
             pk[e] = pack_bf16x2(__fdividef(1.0f, 1.0f + __expf(-g0)),
                                 __fdividef(1.0f, 1.0f + __expf(-g1)));
           }
-          uint4* dst = reinterpret_cast<uint4*>(
-              a.G + (static_cast<long long>(r) * a.N + j) * kHD + h * kD);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
         }
+        // row = lane, 16-byte chunk q at position q ^ ((lane / 2) % 4): conflict-free
+        const int lane = gt & 31;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4*>(stg + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) =
+              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        __syncwarp();
+        __nv_bfloat16* base = part == 0 ? a.Q : part == 1 ? a.K : part == 2 ? a.V : a.G;
+        uint8_t* dst = reinterpret_cast<uint8_t*>(
+            base + ((static_cast<long long>(r) * kHeads + h) * a.N + jw0) * kD);
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          const int off = it * 512 + lane * 16, row = off >> 6, q = (off >> 4) & 3;
+          const uint4 val =
+              *reinterpret_cast<const uint4*>(stg + row * 64 + ((q ^ ((row >> 1) & 3)) << 4));
+          if (jw0 + row < a.N) *reinterpret_cast<uint4*>(dst + off) = val;
+        }
+        __syncwarp();
       }
       tc_fence_before();
       named_barrier_sync(bar_id, kGroupThreads);  // TMEM (and, after the second half, A) reused
@@ -270,6 +313,9 @@ __global__ void __launch_bounds__(kThreads, 1) pair_ln_proj(const ProjArgs a) {
   // ---- teardown: never leave a bulk copy in flight into this CTA's smem
   if (tid == 0 && qkvg && !w_ready) {
     if (!mbar_wait(w_bar, 0, nullptr)) report_status(a.status, kStatusTimeout);
+  }
+  if (mma_thread && z_pending) {
+    if (!mbar_wait(&z_full[grp], z_phase, nullptr)) report_status(a.status, kStatusTimeout);
   }
   tc_fence_before();
   __syncthreads();

@@ -438,8 +438,15 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
     const long long ntiles = static_cast<long long>(nrows) * jtiles;
     const unsigned grid = static_cast<unsigned>(
         std::min<long long>((ntiles + tri::plp::kGroupsPerCta - 1) / tri::plp::kGroupsPerCta, h->num_sms));
+    // Z in boxes of 64 channels x 128 pairs: along j (starting node) or, through
+    // the swapped view, along the rows of Z (ending node)
+    CUtensorMap mz;
+    const uint32_t zb1 = orient == 0 ? 128u : 1u, zb2 = orient == 0 ? 1u : 128u;
+    if (!make_map_3d(&mz, Zb, kCz, N, N, kCz * 2, static_cast<uint64_t>(N) * kCz * 2, 64, zb1,
+                     CU_TENSOR_MAP_SWIZZLE_128B, zb2))
+      return cudaErrorInvalidValue;
     Timer tm(h, st, timed, 0);
-    tri::plp::pair_ln_proj<<<grid, tri::plp::kThreads, tri::plp::kSmemBytes, st>>>(a);
+    tri::plp::pair_ln_proj<<<grid, tri::plp::kThreads, tri::plp::kSmemBytes, st>>>(mz, a);
     return cudaGetLastError();
   };
   if (chunked) CUDA_TRY(proj(0, N, 0, 1));
@@ -473,7 +480,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
       CUDA_TRY(cudaGetLastError());
     }
     {
-      // o, g: this chunk's workspace; z, out: the pair tensor, boxes of 128 pairs
+      // o, g: this chunk's workspace (head-major); z, out: the pair tensor, boxes of 128 pairs
       // along j (starting node) or, through the swapped view, along the rows of Z
       CUtensorMap mo, mg, mz, mout;
       const uint64_t rowb = static_cast<uint64_t>(N) * kCz * 2;
@@ -481,8 +488,8 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
       bool okm =
           make_map_3d(&mo, h->o, kD, N, static_cast<uint64_t>(nr) * kHeads, kD * 2,
                       static_cast<uint64_t>(N) * kD * 2, kD, 128, CU_TENSOR_MAP_SWIZZLE_64B) &&
-          make_map_3d(&mg, h->g, kHD, N, nr, kHD * 2, static_cast<uint64_t>(N) * kHD * 2, 64, 128,
-                      CU_TENSOR_MAP_SWIZZLE_128B) &&
+          make_map_3d(&mg, h->g, kD, N, static_cast<uint64_t>(nr) * kHeads, kD * 2,
+                      static_cast<uint64_t>(N) * kD * 2, kD, 128, CU_TENSOR_MAP_SWIZZLE_64B) &&
           make_map_3d(&mz, Zb, kCz, N, N, kCz * 2, rowb, 64, zb1, CU_TENSOR_MAP_SWIZZLE_128B, zb2) &&
           make_map_3d(&mout, outb, kCz, N, N, kCz * 2, rowb, 64, zb1, CU_TENSOR_MAP_SWIZZLE_128B,
                       zb2);

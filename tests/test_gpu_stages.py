@@ -30,7 +30,7 @@ def _setup(N, orientation, mask="random:0.2", seed=21):
         "q": device_view(ws["q"], (N, 4, N, 32), bf).float(),
         "k": device_view(ws["k"], (N, 4, N, 32), bf).float(),
         "v": device_view(ws["v"], (N, 4, N, 32), bf).float(),
-        "g": device_view(ws["g"], (N, N, 128), bf).float(),
+        "g": device_view(ws["g"], (N, 4, N, 32), bf).float().permute(0, 2, 1, 3).reshape(N, N, 128),
         "o": device_view(ws["o"], (N, 4, N, 32), bf).float(),
         "bias": device_view(ws["bias"], (4, N, ld), bf).float(),
     }
