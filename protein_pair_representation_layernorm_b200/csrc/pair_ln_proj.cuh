@@ -146,50 +146,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       zr[c] = *reinterpret_cast<const uint4*>(sA + (c >> 3) * kAAtomBytes + gt * 128 +
                                               (((c & 7) ^ (gt & 7)) << 4));
 
-    // ---- LayerNorm statistics in fp32 (two passes over registers)
-    float sum = 0.f;
+    // ---- LayerNorm statistics in fp32 (two passes over registers, four
+    // independent partial sums each to keep the dependency chains short)
+    float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
       const uint32_t w[4] = {zr[c].x, zr[c].y, zr[c].z, zr[c].w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sum += bf16lo_to_f32(w[e]) + bf16hi_to_f32(w[e]);
+      for (int e = 0; e < 4; ++e) part[e] += bf16lo_to_f32(w[e]) + bf16hi_to_f32(w[e]);
     }
-    const float mu = sum * (1.0f / kCz);
-    float var = 0.f;
+    const float mu = ((part[0] + part[1]) + (part[2] + part[3])) * (1.0f / kCz);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) part[e] = 0.f;
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
       const uint32_t w[4] = {zr[c].x, zr[c].y, zr[c].z, zr[c].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float d0 = bf16lo_to_f32(w[e]) - mu, d1 = bf16hi_to_f32(w[e]) - mu;
-        var = fmaf(d0, d0, var);
-        var = fmaf(d1, d1, var);
+        part[e] = fmaf(d0, d0, part[e]);
+        part[e] = fmaf(d1, d1, part[e]);
       }
     }
+    const float var = (part[0] + part[1]) + (part[2] + part[3]);
     const float rstd = rsqrtf(var * (1.0f / kCz) + a.eps);
 
-    // ---- normalise, bias dot products, bf16 A tile
+    // ---- normalise, bias dot products, bf16 A tile (parameters read as float4)
     float bacc[kHeads] = {0.f, 0.f, 0.f, 0.f};
+    const float4* g4 = reinterpret_cast<const float4*>(s_gamma);
+    const float4* b4 = reinterpret_cast<const float4*>(s_beta);
+    const float4* w4 = reinterpret_cast<const float4*>(s_wb);
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
       const uint32_t w[4] = {zr[c].x, zr[c].y, zr[c].z, zr[c].w};
-      uint32_t packed[4];
+      float xv[8];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int ch = c * 8 + 2 * e;
-        const float x0 = (bf16lo_to_f32(w[e]) - mu) * rstd * s_gamma[ch] + s_beta[ch];
-        const float x1 = (bf16hi_to_f32(w[e]) - mu) * rstd * s_gamma[ch + 1] + s_beta[ch + 1];
+      for (int hq = 0; hq < 2; ++hq) {
+        const float4 gm = g4[2 * c + hq], bt = b4[2 * c + hq];
+        xv[4 * hq + 0] = (bf16lo_to_f32(w[2 * hq]) - mu) * rstd * gm.x + bt.x;
+        xv[4 * hq + 1] = (bf16hi_to_f32(w[2 * hq]) - mu) * rstd * gm.y + bt.y;
+        xv[4 * hq + 2] = (bf16lo_to_f32(w[2 * hq + 1]) - mu) * rstd * gm.z + bt.z;
+        xv[4 * hq + 3] = (bf16hi_to_f32(w[2 * hq + 1]) - mu) * rstd * gm.w + bt.w;
+      }
 #pragma unroll
-        for (int h = 0; h < kHeads; ++h) {
-          bacc[h] = fmaf(s_wb[h * kCz + ch], x0, bacc[h]);
-          bacc[h] = fmaf(s_wb[h * kCz + ch + 1], x1, bacc[h]);
-        }
-        packed[e] = pack_bf16x2(x0, x1);
+      for (int h = 0; h < kHeads; ++h) {
+        const float4 wa = w4[(h * kCz) / 4 + 2 * c], wb = w4[(h * kCz) / 4 + 2 * c + 1];
+        float acc2 = bacc[h];
+        acc2 = fmaf(wa.x, xv[0], acc2);
+        acc2 = fmaf(wa.y, xv[1], acc2);
+        acc2 = fmaf(wa.z, xv[2], acc2);
+        acc2 = fmaf(wa.w, xv[3], acc2);
+        acc2 = fmaf(wb.x, xv[4], acc2);
+        acc2 = fmaf(wb.y, xv[5], acc2);
+        acc2 = fmaf(wb.z, xv[6], acc2);
+        acc2 = fmaf(wb.w, xv[7], acc2);
+        bacc[h] = acc2;
       }
       if (qkvg) {
         // K-major, 128 B swizzle: row gt, 16-byte chunk (c % 8) of K-slab c / 8
         uint8_t* dst = sA + (c >> 3) * kAAtomBytes + gt * 128 + (((c & 7) ^ (gt & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        *reinterpret_cast<uint4*>(dst) =
+            make_uint4(pack_bf16x2(xv[0], xv[1]), pack_bf16x2(xv[2], xv[3]),
+                       pack_bf16x2(xv[4], xv[5]), pack_bf16x2(xv[6], xv[7]));
       }
     }
     if (a.write_bias) {
@@ -260,11 +278,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // and writes it back with 512-byte coalesced stores.
       const int jw0 = static_cast<int>(tile % jtiles) * kTileM + (warp & 3) * 32;
       uint8_t* stg = smem + kSmemStg + warp * kStgBytes;
+      uint32_t v[32], vn[32];
+      tmem_ld32(tmem + lane_base, vn);
 #pragma unroll 1
       for (int cc = 0; cc < 8; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + cc * 32, v);
         tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = vn[e];
+        if (cc + 1 < 8) tmem_ld32(tmem + lane_base + (cc + 1) * 32, vn);  // overlap the next load
         const int part = half * 2 + (cc >> 2), h = cc & 3;
         uint32_t pk[16];
         if (part < 3) {
@@ -273,12 +294,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 16; ++e)
             pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
         } else {
+          // sigmoid(t) = 1/2 + tanh(t/2)/2: one special-function op per value
+          const float4* bg4 = reinterpret_cast<const float4*>(s_bg + h * kD);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float g0 = __uint_as_float(v[2 * e]) + s_bg[h * kD + 2 * e];
-            const float g1 = __uint_as_float(v[2 * e + 1]) + s_bg[h * kD + 2 * e + 1];
-            pk[e] = pack_bf16x2(__fdividef(1.0f, 1.0f + __expf(-g0)),
-                                __fdividef(1.0f, 1.0f + __expf(-g1)));
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 bb = bg4[e4];
+            const float t0 = __uint_as_float(v[4 * e4]) + bb.x;
+            const float t1 = __uint_as_float(v[4 * e4 + 1]) + bb.y;
+            const float t2 = __uint_as_float(v[4 * e4 + 2]) + bb.z;
+            const float t3 = __uint_as_float(v[4 * e4 + 3]) + bb.w;
+            pk[2 * e4] = pack_bf16x2(fmaf(0.5f, tanh_approx(0.5f * t0), 0.5f),
+                                     fmaf(0.5f, tanh_approx(0.5f * t1), 0.5f));
+            pk[2 * e4 + 1] = pack_bf16x2(fmaf(0.5f, tanh_approx(0.5f * t2), 0.5f),
+                                         fmaf(0.5f, tanh_approx(0.5f * t3), 0.5f));
           }
         }
         // row = lane, 16-byte chunk q at position q ^ ((lane / 2) % 4): conflict-free
