@@ -14,12 +14,15 @@
 // The 3 rows share every bias tile b_h(j0.., k-tile), which is loaded once per
 // CTA; K and V differ per row.
 //
-// Warp roles (448 threads, at most four warps per SM sub-partition, so up to
-// 128 registers per thread):
+// Warp roles (512 threads, four warps per SM sub-partition, so up to 128
+// registers per thread):
 //   warps 4r..4r+3  softmax group r = row i0+r (thread = query j = TMEM lane j)
 //   warp 12         TMA producer: Q once; per key tile K, V of the 3 rows + the bias tile
-//   warp 13         MMA issuer (one thread): S = Q K^T (M=128, N=64, K=32) and
-//                   O += P V (M=128, N=32, K=64, P read from TMEM)
+//   warp 13+r       MMA issuer of row r (one thread): S_r = Q_r K_r^T (M=128, N=64,
+//                   K=32) and O_r += P_r V_r (M=128, N=32, K=64, P read from TMEM)
+// One issuing thread per row keeps each issuer's instruction stream short (it
+// shares a sub-partition with three softmax warps, and the tensor core waits
+// on it) and lets a row's MMAs go ahead without waiting for the other rows.
 // TMEM (512 columns): per row two S/P buffers of 64 columns at 128r and 128r+64
 // (fp32 scores; bf16 P aliased over the first 32 columns of its buffer), O_r at
 // 384 + 32r.
@@ -55,9 +58,9 @@ constexpr int kBK = 64;           // keys per step
 constexpr int kRows = 3;          // problem rows per CTA
 constexpr int kGroups = kRows;    // softmax warpgroups, one row each
 constexpr int kStages = 4;
-constexpr int kThreads = (4 * kGroups + 2) * 32;
+constexpr int kThreads = (4 * kGroups + 1 + kGroups) * 32;
 constexpr int kProducerWarp = 4 * kGroups;
-constexpr int kMmaWarp = 4 * kGroups + 1;
+constexpr int kMmaWarp0 = 4 * kGroups + 1;  // MMA warp of row g: kMmaWarp0 + g
 constexpr float kTau = 8.0f;
 constexpr float kFloor = -1.0e30f;
 
@@ -71,8 +74,8 @@ constexpr uint32_t kStageBytes = kStageB + kBiasTileBytes;  // 40960
 constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemStages = kRows * kQTileBytes;       // 24576
 constexpr uint32_t kSmemBar = kSmemStages + kStages * kStageBytes;
-// q_full, st_full[S], st_empty[S], s_full[R][2], p_full[R][2], o_ready[R], o_full, drain
-constexpr uint32_t kNumBars = 1 + 2 * kStages + 2 * kGroups + 2 * kGroups + kGroups + 2;
+// q_full, st_full[S], st_empty[S], s_full[R][2], p_full[R][2], o_ready[R], o_full[R], drain[R]
+constexpr uint32_t kNumBars = 1 + 2 * kStages + 2 * kGroups + 2 * kGroups + 3 * kGroups;
 constexpr uint32_t kSmemBytes = kSmemBar + kNumBars * 8 + 16 + 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;      // + 128 r + 64 b
@@ -97,9 +100,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // still works on tile t; with a single barrier that early arrival would count
   // towards tile t's phase.
   uint64_t* p_full = s_full + 2 * kGroups;  // [g][buffer]
-  uint64_t* o_ready = p_full + 2 * kGroups;  // PV(T-2) of row g complete
-  uint64_t* o_full = o_ready + kGroups;
-  uint64_t* drain = o_full + 1;
+  uint64_t* o_ready = p_full + 2 * kGroups;  // [g]: PV(T-2) of row g complete
+  uint64_t* o_full = o_ready + kGroups;      // [g]: every MMA of row g complete
+  uint64_t* drain = o_full + kGroups;        // [g]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -114,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&st_full[s], 1);
-      mbar_init(&st_empty[s], 1 + kGroups * 4);  // MMA commit + one arrive per softmax warp
+      mbar_init(&st_empty[s], kGroups + kGroups * 4);  // one commit per MMA warp, one arrive per softmax warp
     }
     for (int g = 0; g < kGroups; ++g) {
       mbar_init(&s_full[2 * g], 1);
@@ -122,13 +125,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[2 * g], 4);
       mbar_init(&p_full[2 * g + 1], 4);
       mbar_init(&o_ready[g], 1);
+      mbar_init(&o_full[g], 1);
+      mbar_init(&drain[g], 1);
     }
-    mbar_init(o_full, 1);
-    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kMmaWarp0) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -182,8 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp >= kMmaWarp0) {
+    // ------------------------------------------------------------ MMA issuer of row g
+    const int g = warp - kMmaWarp0;
     if (lane == 0) {
       constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kBK, false);
       constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kD, true);
@@ -193,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // carries into the rest).  The tile loop below is unrolled over the
       // kStages stages so that stage, S buffer, barrier parities and operand
       // offsets are compile-time constants: this thread's instruction issue is
-      // on the critical path of the whole CTA.
+      // on the critical path of its row.
       const uint64_t dQ = smem_desc(smem_u32(smem + kSmemQ), 512, kSwizzle64B);
       const uint64_t dSt = smem_desc(smem_u32(smem + kSmemStages), 512, kSwizzle64B);
       const uint32_t q_lo = static_cast<uint32_t>(dQ), st_lo = static_cast<uint32_t>(dSt);
@@ -201,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto qdesc = [&](uint32_t off) { return q_hi | (q_lo + (off >> 4)); };
       auto sdesc = [&](uint32_t off) { return st_hi | (st_lo + (off >> 4)); };
       // S(g) = Q_g K_g^T from stage `st` into S buffer `b` of row g
-      auto issue_qk = [&](int g, int st, int b) {
+      auto issue_qk = [&](int st, int b) {
         const uint32_t dS = tmem + kColS + 128 * g + 64 * b;
 #pragma unroll
         for (int kc = 0; kc < kD / 16; ++kc)
@@ -218,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok || t >= T) break;
         if (!(ok = mbar_wait(&st_full[t], 0, abort_flag))) break;
         tc_fence_after();
-        for (int g = 0; g < kGroups; ++g) issue_qk(g, t, t);
+        issue_qk(t, t);
         issued = true;
       }
       for (int base = 0; ok && base < T; base += kStages) {
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t pb = (s >> 1) & 1;              // (t / 2) % 2
           const int s2 = (s + 2) % kStages;              // stage of tile t+2
           const uint32_t ph2 = s + 2 < kStages ? ph : ph ^ 1u;
-          for (int g = 0; g < kGroups; ++g) {
+          {
             if (!(ok = mbar_wait(&p_full[2 * g + b], pb, abort_flag))) break;
             tc_fence_after();
             // O_g += P_g(t) V_g(t), P read from S buffer t % 2
@@ -245,25 +249,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             // reads it); its commit also tells the softmax that PV(t) is
             // complete.  After the last QK, o_ready carries that signal.
             if (t + 2 < T) {
-              if (g == 0 && !(ok = mbar_wait(&st_full[s2], ph2, abort_flag))) break;
+              if (!(ok = mbar_wait(&st_full[s2], ph2, abort_flag))) break;
               tc_fence_after();
-              issue_qk(g, s2, b);
+              issue_qk(s2, b);
             } else if (t + 2 == T) {
               mma_commit(&o_ready[g]);
             }
+            mma_commit(&st_empty[s]);  // this row's MMAs on stage s
           }
-          if (!ok) break;
-          mma_commit(&st_empty[s]);
         }
       }
       if (ok) {
-        mma_commit(o_full);
+        mma_commit(&o_full[g]);
       } else {
         *abort_flag = 1;
         report_status(a.status, kStatusTimeout);
-        if (issued) {  // wait until no MMA of this CTA is in flight
-          mma_commit(drain);
-          mbar_wait(drain, 0, nullptr);
+        if (issued) {  // wait until no MMA of this warp is in flight
+          mma_commit(&drain[g]);
+          mbar_wait(&drain[g], 0, nullptr);
         }
       }
     }
@@ -369,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&p_full[2 * g + (t & 1)]);
     }
     // ---- epilogue: o = O / l
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_full[g], 0, abort_flag));
     if (ok) {
       tc_fence_after();
       const int j = j0 + jl;
@@ -397,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kMmaWarp0) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
