@@ -49,7 +49,7 @@ DATASHEET_BF16_TFLOPS = 2250.0
 # DRAM bytes per tri_attn_fwd launch (starting node, N = 1536) from one ncu
 # capture (profiles/tri_attn_fwd_N1536.md), valid only for the kernel source
 # with this hash; otherwise reported as null.
-TRAFFIC = {"tri_attn_fwd.cuh": "7420e4509ec70df7", "bytes_per_launch": 1.83e9 + 0.58581e9}
+TRAFFIC = {"tri_attn_fwd.cuh": "eb080b79a171320f", "bytes_per_launch": 1.831321e9 + 0.584901e9}
 
 
 def parse():
