@@ -161,9 +161,9 @@ int tri_attn_debug_workspace(tri_attn_handle *h, void **q, void **k, void **v, v
  * status word and the workspace) lives in one statically allocated device array
  * of 32 MiB inside this library; every GPU that loads the library holds it
  * until the process exits.  Rows are processed in chunks that fit the array.
- * Sizes it cannot hold (the whole logit bias plus one four-row chunk must fit,
- * which allows N up to about 1750) return TRI_ATTN_ERR_UNSUPPORTED before
- * anything is launched.  The first call on a device also looks up the array's
+ * Sizes it cannot hold (the whole logit bias plus one three-row chunk must fit,
+ * which allows N up to 1792) return TRI_ATTN_ERR_UNSUPPORTED before anything
+ * is launched.  The first call on a device also looks up the array's
  * device address (cudaGetSymbolAddress); make that first call before any stream
  * capture.  All calls share the one array, which keeps the last call's contents
  * (the status word is cleared at the start of each call): calls that overlap on
