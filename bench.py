@@ -45,6 +45,9 @@ WORKLOAD = 3
 METRIC = "triangle-attn TFLOP/s at N=1536 bf16; % of B200 bf16 dense tensor peak"
 UNIT = "TFLOP/s"
 DATASHEET_BF16_TFLOPS = 2250.0
+EX2_PER_CLK_SM = 16      # special-function unit exp2 rate, measured with a probe on the B200
+NUM_SMS = 148
+SM_MAX_MHZ = 1965.0
 
 # DRAM bytes per tri_attn_fwd launch (starting node, N = 1536) from one ncu
 # capture (profiles/tri_attn_fwd_N1536.md), valid only for the kernel source
@@ -255,6 +258,7 @@ def run_ours(args, world, rank, local):
     n_valid = N if inp.mask is None else int(inp.mask.sum())
     H, d = 4, 32
     flops_attn = 4.0 * N * N * n_valid * H * d          # one orientation
+    exps_attn = float(N) * N * n_valid * H                # one exp2 per score
     flops_step = 2 * flops_attn
     blk = binding.TriangleAttention(inp.weights(), dtype=torch.bfloat16)
     st = torch.cuda.Stream()
@@ -348,7 +352,17 @@ def run_ours(args, world, rank, local):
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": attn_tf / peak_tf,
                      "peak_source": f"{peak_src} bf16_tflops (burst)", "traffic": traffic,
                      "algorithmic_flops_per_launch": flops_attn,
-                     "launch_ms": attn_ms},
+                     "launch_ms": attn_ms,
+                     # what actually limits the kernel: one exp2 per score on the
+                     # special-function unit, 16 per clock per SM (measured with a
+                     # probe), at the maximum SM clock
+                     "limiter": {"unit_name": "exp2 (special-function unit)",
+                                 "achieved": exps_attn / (attn_ms / 1e3),
+                                 "peak": EX2_PER_CLK_SM * NUM_SMS * SM_MAX_MHZ * 1e6,
+                                 "unit": "ex2/s",
+                                 "frac": exps_attn / (attn_ms / 1e3)
+                                 / (EX2_PER_CLK_SM * NUM_SMS * SM_MAX_MHZ * 1e6),
+                                 "peak_derivation": "16 ex2/clk/SM x 148 SMs x 1965 MHz"}},
         "kernels": {
             "pair_ln_proj": {"ms": proj_ms, "launches": kn[0],
                              "GB/s": proj_bytes / (proj_ms / 1e3) / 1e9,
