@@ -268,12 +268,13 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// 2^x for two values on the FMA pipe (x <= 64; results below 2^-126 flush to 0,
-// x = -inf gives exactly 0).  Cody-Waite style reduction x = n + f with
+// 2^x for two values on the FMA pipe (x <= 64; relative error 7.5e-5 while the
+// result is a normal float, x >= -125; a value in [0, 2^-125] down to x = -127
+// and exactly 0 below, -inf included).  Cody-Waite style reduction x = n + f with
 // n = round(x), |f| <= 1/2: n is read from the low mantissa bits of x + 1.5 * 2^23.
-// 2^f is a degree-3 polynomial whose coefficients were fitted for minimal
-// relative error on [-1/2, 1/2] (iteratively reweighted least squares, max
-// relative error 7.5e-5); 2^n is applied by adding n to the exponent field, and
+// 2^f is the degree-3 polynomial of minimal maximum relative error on
+// [-1/2, 1/2] (Remez exchange, csrc/fit_exp2_poly.py; max relative error
+// 7.5e-5); 2^n is applied by adding n to the exponent field, and
 // a result whose exponent would underflow (the sum turns negative) is clamped to 0.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
@@ -281,10 +282,10 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   const float2 t = __fadd2_rn(xc, make_float2(kRound, kRound));
   const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
   const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), xc);
-  float2 p = __ffma2_rn(f, make_float2(0.05517132f, 0.05517132f),
-                        make_float2(0.24261054f, 0.24261054f));
-  p = __ffma2_rn(p, f, make_float2(0.69326097f, 0.69326097f));
-  p = __ffma2_rn(p, f, make_float2(0.99992812f, 0.99992812f));
+  float2 p = __ffma2_rn(f, make_float2(0.05517167f, 0.05517167f),
+                        make_float2(0.24261112f, 0.24261112f));
+  p = __ffma2_rn(p, f, make_float2(0.69326099f, 0.69326099f));
+  p = __ffma2_rn(p, f, make_float2(0.99992807f, 0.99992807f));
   const int a = max(__float_as_int(p.x) + (__float_as_int(t.x) << 23), 0);
   const int b = max(__float_as_int(p.y) + (__float_as_int(t.y) << 23), 0);
   return make_float2(__int_as_float(a), __int_as_float(b));
