@@ -46,22 +46,6 @@ constexpr uint32_t kNumBars = 1 + 3 * kStages;
 constexpr uint32_t kSmemBytes = kSmemBar + kNumBars * 8 + 16 + 1024;
 constexpr uint32_t kTmemCols = 256;  // two 128-column accumulators
 
-// TMA store of a box from shared memory (bulk-group completion).
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0,
-                                             int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_read_all() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     gate_out(const __grid_constant__ CUtensorMap map_o, const __grid_constant__ CUtensorMap map_g,
              const __grid_constant__ CUtensorMap map_z, const __grid_constant__ CUtensorMap map_out,

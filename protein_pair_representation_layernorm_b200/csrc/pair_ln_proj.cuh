@@ -18,9 +18,9 @@
 // N = 256 (q|k, then v|g), W = [Wq; Wk; Wv; Wg] resident in shared memory for the
 // whole kernel, each half accumulating in fp32 in the group's 256 TMEM columns.
 // Each thread reads back its TMEM lane; q (scaled by log2(e)/sqrt(d)), k, v and
-// sigmoid(g + bg) are written head-major ([rows][H][N][d], bf16), each warp
-// staging its 32 pairs' 64-byte rows in shared memory so that the global stores
-// are contiguous 512-byte blocks.  While one group runs its MMAs the other normalises or
+// sigmoid(g + bg) are written head-major ([rows][H][N][d], bf16): each warp
+// stages its 32 pairs' 64-byte rows of one head in shared memory and writes
+// them with one TMA store (a contiguous 2 KB block).  While one group runs its MMAs the other normalises or
 // stores, so the tensor core, the ALUs and HBM overlap.
 //
 // This is the HBM-bound step: per pair it reads 256 B and writes 1 KB + 8 B.
@@ -53,7 +53,9 @@ static_assert(kGroupsPerCta * 2 * 8 + 8 + 8 <= 64, "barrier area");
 constexpr uint32_t kTmemCols = 512;                                     // 256 per group
 
 __global__ void __launch_bounds__(kThreads, 1)
-    pair_ln_proj(const __grid_constant__ CUtensorMap map_z, const ProjArgs a) {
+    pair_ln_proj(const __grid_constant__ CUtensorMap map_z, const __grid_constant__ CUtensorMap map_q,
+                 const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                 const __grid_constant__ CUtensorMap map_g, const ProjArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -146,68 +148,70 @@ __global__ void __launch_bounds__(kThreads, 1)
       zr[c] = *reinterpret_cast<const uint4*>(sA + (c >> 3) * kAAtomBytes + gt * 128 +
                                               (((c & 7) ^ (gt & 7)) << 4));
 
-    // ---- LayerNorm statistics in fp32 (two passes over registers, four
-    // independent partial sums each to keep the dependency chains short)
-    float part[4] = {0.f, 0.f, 0.f, 0.f};
+    // ---- LayerNorm statistics in fp32: two passes over registers, packed
+    // fp32x2 arithmetic on channel pairs, two independent accumulators each
+    auto chan2 = [](uint32_t w) { return make_float2(bf16lo_to_f32(w), bf16hi_to_f32(w)); };
+    float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
-      const uint32_t w[4] = {zr[c].x, zr[c].y, zr[c].z, zr[c].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) part[e] += bf16lo_to_f32(w[e]) + bf16hi_to_f32(w[e]);
+      acc[0] = __fadd2_rn(acc[0], chan2(zr[c].x));
+      acc[1] = __fadd2_rn(acc[1], chan2(zr[c].y));
+      acc[0] = __fadd2_rn(acc[0], chan2(zr[c].z));
+      acc[1] = __fadd2_rn(acc[1], chan2(zr[c].w));
     }
-    const float mu = ((part[0] + part[1]) + (part[2] + part[3])) * (1.0f / kCz);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) part[e] = 0.f;
+    const float mu = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) * (1.0f / kCz);
+    const float2 nmu = make_float2(-mu, -mu);
+    acc[0] = acc[1] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
       const uint32_t w[4] = {zr[c].x, zr[c].y, zr[c].z, zr[c].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float d0 = bf16lo_to_f32(w[e]) - mu, d1 = bf16hi_to_f32(w[e]) - mu;
-        part[e] = fmaf(d0, d0, part[e]);
-        part[e] = fmaf(d1, d1, part[e]);
+        const float2 d = __fadd2_rn(chan2(w[e]), nmu);
+        acc[e & 1] = __ffma2_rn(d, d, acc[e & 1]);
       }
     }
-    const float var = (part[0] + part[1]) + (part[2] + part[3]);
+    const float var = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
     const float rstd = rsqrtf(var * (1.0f / kCz) + a.eps);
+    const float2 rstd2 = make_float2(rstd, rstd);
 
-    // ---- normalise, bias dot products, bf16 A tile (parameters read as float4)
-    float bacc[kHeads] = {0.f, 0.f, 0.f, 0.f};
+    // ---- normalise, bias dot products, bf16 A tile (parameters read as float4,
+    // arithmetic on channel pairs)
+    float2 bacc[kHeads] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                           make_float2(0.f, 0.f)};
     const float4* g4 = reinterpret_cast<const float4*>(s_gamma);
     const float4* b4 = reinterpret_cast<const float4*>(s_beta);
     const float4* w4 = reinterpret_cast<const float4*>(s_wb);
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
       const uint32_t w[4] = {zr[c].x, zr[c].y, zr[c].z, zr[c].w};
-      float xv[8];
+      float2 xv[4];  // channels 8c .. 8c+7 as pairs
 #pragma unroll
       for (int hq = 0; hq < 2; ++hq) {
         const float4 gm = g4[2 * c + hq], bt = b4[2 * c + hq];
-        xv[4 * hq + 0] = (bf16lo_to_f32(w[2 * hq]) - mu) * rstd * gm.x + bt.x;
-        xv[4 * hq + 1] = (bf16hi_to_f32(w[2 * hq]) - mu) * rstd * gm.y + bt.y;
-        xv[4 * hq + 2] = (bf16lo_to_f32(w[2 * hq + 1]) - mu) * rstd * gm.z + bt.z;
-        xv[4 * hq + 3] = (bf16hi_to_f32(w[2 * hq + 1]) - mu) * rstd * gm.w + bt.w;
+        const float2 d0 = __fadd2_rn(chan2(w[2 * hq]), nmu);
+        const float2 d1 = __fadd2_rn(chan2(w[2 * hq + 1]), nmu);
+        xv[2 * hq] = __ffma2_rn(__fmul2_rn(d0, rstd2), make_float2(gm.x, gm.y),
+                                make_float2(bt.x, bt.y));
+        xv[2 * hq + 1] = __ffma2_rn(__fmul2_rn(d1, rstd2), make_float2(gm.z, gm.w),
+                                    make_float2(bt.z, bt.w));
       }
 #pragma unroll
       for (int h = 0; h < kHeads; ++h) {
         const float4 wa = w4[(h * kCz) / 4 + 2 * c], wb = w4[(h * kCz) / 4 + 2 * c + 1];
-        float acc2 = bacc[h];
-        acc2 = fmaf(wa.x, xv[0], acc2);
-        acc2 = fmaf(wa.y, xv[1], acc2);
-        acc2 = fmaf(wa.z, xv[2], acc2);
-        acc2 = fmaf(wa.w, xv[3], acc2);
-        acc2 = fmaf(wb.x, xv[4], acc2);
-        acc2 = fmaf(wb.y, xv[5], acc2);
-        acc2 = fmaf(wb.z, xv[6], acc2);
-        acc2 = fmaf(wb.w, xv[7], acc2);
+        float2 acc2 = bacc[h];
+        acc2 = __ffma2_rn(make_float2(wa.x, wa.y), xv[0], acc2);
+        acc2 = __ffma2_rn(make_float2(wa.z, wa.w), xv[1], acc2);
+        acc2 = __ffma2_rn(make_float2(wb.x, wb.y), xv[2], acc2);
+        acc2 = __ffma2_rn(make_float2(wb.z, wb.w), xv[3], acc2);
         bacc[h] = acc2;
       }
       if (qkvg) {
         // K-major, 128 B swizzle: row gt, 16-byte chunk (c % 8) of K-slab c / 8
         uint8_t* dst = sA + (c >> 3) * kAAtomBytes + gt * 128 + (((c & 7) ^ (gt & 7)) << 4);
         *reinterpret_cast<uint4*>(dst) =
-            make_uint4(pack_bf16x2(xv[0], xv[1]), pack_bf16x2(xv[2], xv[3]),
-                       pack_bf16x2(xv[4], xv[5]), pack_bf16x2(xv[6], xv[7]));
+            make_uint4(pack_bf16x2(xv[0].x, xv[0].y), pack_bf16x2(xv[1].x, xv[1].y),
+                       pack_bf16x2(xv[2].x, xv[2].y), pack_bf16x2(xv[3].x, xv[3].y));
       }
     }
     if (a.write_bias) {
@@ -216,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int h = 0; h < kHeads; ++h)
           a.bias[(static_cast<long long>(h) * a.N + i) * a.ld_bias + j] =
-              __float2bfloat16_rn(key_valid ? bacc[h] : kMaskedLogit);
+              __float2bfloat16_rn(key_valid ? bacc[h].x + bacc[h].y : kMaskedLogit);
       }
     }
     if (!qkvg) {
@@ -309,24 +313,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          fmaf(0.5f, tanh_approx(0.5f * t3), 0.5f));
           }
         }
-        // row = lane, 16-byte chunk q at position q ^ ((lane / 2) % 4): conflict-free
+        // The staging buffer is the 64-byte-swizzled image of a 32 x 32 bf16 TMA
+        // box (row = lane, 16-byte chunk q at position q ^ ((lane / 2) % 4), which
+        // is also conflict-free); lane 0 stores it with one TMA store, which
+        // clips the rows past N.  The previous chunk's store must have read the
+        // buffer before it is rewritten.
         const int lane = gt & 31;
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           *reinterpret_cast<uint4*>(stg + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) =
               make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        fence_proxy_async_smem();
         __syncwarp();
-        __nv_bfloat16* base = part == 0 ? a.Q : part == 1 ? a.K : part == 2 ? a.V : a.G;
-        uint8_t* dst = reinterpret_cast<uint8_t*>(
-            base + ((static_cast<long long>(r) * kHeads + h) * a.N + jw0) * kD);
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-          const int off = it * 512 + lane * 16, row = off >> 6, q = (off >> 4) & 3;
-          const uint4 val =
-              *reinterpret_cast<const uint4*>(stg + row * 64 + ((q ^ ((row >> 1) & 3)) << 4));
-          if (jw0 + row < a.N) *reinterpret_cast<uint4*>(dst + off) = val;
+        if (lane == 0) {
+          const CUtensorMap* m = part == 0 ? &map_q : part == 1 ? &map_k : part == 2 ? &map_v : &map_g;
+          tma_store_3d(m, stg, 0, jw0, r * kHeads + h);
+          bulk_commit();
         }
-        __syncwarp();
       }
       tc_fence_before();
       named_barrier_sync(bar_id, kGroupThreads);  // TMEM (and, after the second half, A) reused
@@ -338,7 +343,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // ---- teardown: never leave a bulk copy in flight into this CTA's smem
+  // ---- teardown: no bulk copy may still be reading or writing this CTA's smem
+  if ((gt & 31) == 0) bulk_wait_all();
   if (tid == 0 && qkvg && !w_ready) {
     if (!mbar_wait(w_bar, 0, nullptr)) report_status(a.status, kStatusTimeout);
   }

@@ -445,8 +445,18 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
     if (!make_map_3d(&mz, Zb, kCz, N, N, kCz * 2, static_cast<uint64_t>(N) * kCz * 2, 64, zb1,
                      CU_TENSOR_MAP_SWIZZLE_128B, zb2))
       return cudaErrorInvalidValue;
+    // q, k, v, g outputs ([rows][H][N][d] bf16): 32 x 32 boxes, 64 B swizzle (the
+    // kernel's per-warp staging layout); a bias-only pass never stores through them
+    CUtensorMap mo[4];
+    void* outs[4] = {h->q, h->k, h->v, h->g};
+    const uint64_t rh = static_cast<uint64_t>(wq ? nrows : 1) * kHeads;
+    for (int m = 0; m < 4; ++m)
+      if (!make_map_3d(&mo[m], outs[m], kD, N, rh, kD * 2, static_cast<uint64_t>(N) * kD * 2, kD,
+                       32, CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
     Timer tm(h, st, timed, 0);
-    tri::plp::pair_ln_proj<<<grid, tri::plp::kThreads, tri::plp::kSmemBytes, st>>>(mz, a);
+    tri::plp::pair_ln_proj<<<grid, tri::plp::kThreads, tri::plp::kSmemBytes, st>>>(
+        mz, mo[0], mo[1], mo[2], mo[3], a);
     return cudaGetLastError();
   };
   if (chunked) CUDA_TRY(proj(0, N, 0, 1));
