@@ -81,7 +81,10 @@ def test_workload4_sampled(orientation):
     _check_lines(inp, orientation, lines, "bf16", f"workload 4 orient {orientation}")
 
 
-@pytest.mark.parametrize("N", [1, 7, 97, 130, 200])
+# key-tile counts T = ceil(N / 64): 1, 1, 2, 3, 4, 5, 7 (the attention kernel's
+# issue loops are unrolled over its 4 stages: 300 and 420 end one and three
+# tiles into a second round); query tiles of 128 are ragged for all but N = 1
+@pytest.mark.parametrize("N", [1, 7, 97, 130, 200, 300, 420])
 @pytest.mark.parametrize("orientation", [0, 1])
 def test_ragged_sizes(N, orientation):
     inp = workloads.make_inputs(N, "bf16", 100 + N, "random:0.15" if N > 1 else "none")
