@@ -145,6 +145,45 @@ size_t tri_attn_workspace_bytes(tri_attn_dtype dtype, int N);
 int tri_attn_debug_workspace(tri_attn_handle *h, void **q, void **k, void **v, void **g,
                              void **bias, void **o, int *ld_bias, int *rows);
 
+/* ---- row-sharded execution (bf16) -----------------------------------------
+ *
+ * A starting-node block splits over devices by problem rows i: row i needs
+ * only its own K and V (pairs (i, k)) plus the logit bias of every pair, so a
+ * device that holds the row slab Z[row0 .. row0+nrows-1][0..N-1][c_z] can
+ * compute those output rows once the whole bias is known (the 1D row sharding
+ * of the Design-CP technical summary, §Metodología 1, with the bias as the one
+ * exchanged quantity).  The caller runs the exchange between the two calls:
+ *
+ *   1. tri_attn_rows_bias: the slab's bias rows, bias_rows[h][r][k] for the
+ *      problem rows row0+r, heads h, keys k < ld (ld = tri_attn_bias_ld(N));
+ *   2. gather every device's rows into bias_all[h][i][k] ([H][N][ld]);
+ *   3. tri_attn_rows_forward: the block on the slab, reading bias_all.
+ *
+ * An ending-node block is the starting-node block of the transposed pair
+ * tensor (pair (i, j) -> (j, i)): shard its rows, i.e. the columns of Z.
+ * Bias values: bf16, already scaled by log2(e), -3e38 at masked keys and at
+ * k >= N.  Results are bitwise identical to tri_attn_forward on the whole
+ * tensor.  These calls are asynchronous on `stream` like tri_attn_forward
+ * (TRI_ATTN_FLAG_SYNC and TRI_ATTN_FLAG_TIME_KERNELS apply), need a BF16
+ * handle (else TRI_ATTN_ERR_UNSUPPORTED) and device pointers aligned to 16
+ * bytes; mask is the whole [N] key mask.  Z_rows and out_rows are
+ * [nrows][N][c_z]; out_rows may equal Z_rows, any other overlap returns
+ * TRI_ATTN_ERR_ALIAS.  Invalid row ranges return TRI_ATTN_ERR_INVALID_ARG. */
+
+/* Row length (elements) of the logit-bias buffers for a problem of size N:
+ * N rounded up to a multiple of 64; 0 for N < 1. */
+int tri_attn_bias_ld(int N);
+
+/* Phase 1: bias_rows ([H][nrows][ld] bf16, device) for the slab's rows. */
+int tri_attn_rows_bias(tri_attn_handle *h, const void *Z_rows, int N, int row0, int nrows,
+                       const uint8_t *mask, void *bias_rows, void *stream, unsigned flags);
+
+/* Phase 3: out_rows = the starting-node block on the slab, with bias_all
+ * ([H][N][ld] bf16, device) the whole problem's logit bias. */
+int tri_attn_rows_forward(tri_attn_handle *h, const void *Z_rows, int N, int row0, int nrows,
+                          const uint8_t *mask, const void *bias_all, void *out_rows,
+                          void *stream, unsigned flags);
+
 /* One forward of the bf16 block that allocates no device memory at all.
  *
  * For callers that are not allowed to call cudaMalloc: code embedded in a host

@@ -88,6 +88,9 @@ def lib() -> ctypes.CDLL:
             ctypes.POINTER(ci), ctypes.POINTER(ci)]
         L.tri_attn_forward_noalloc.argtypes = [ctypes.POINTER(tri_attn_params), vp, ci, vp, ci,
                                                vp, vp, cu]
+        L.tri_attn_bias_ld.argtypes = [ci]
+        L.tri_attn_rows_bias.argtypes = [vp, vp, ci, ci, ci, vp, vp, vp, cu]
+        L.tri_attn_rows_forward.argtypes = [vp, vp, ci, ci, ci, vp, vp, vp, vp, cu]
         L.tri_attn_destroy.argtypes = [vp]
         L.tri_attn_status_string.argtypes = [ci]
         L.tri_attn_status_string.restype = ctypes.c_char_p
@@ -239,6 +242,45 @@ class TriangleAttention:
                                    list(orientations), _ptr(out), _stream_handle(stream), flags)
         if rc != TRI_ATTN_OK:
             raise TriAttnError(rc, "tri_attn_forward_host")
+        return out
+
+    # ---- row-sharded execution (bf16): see tri_attn_rows_bias / _forward in
+    # include/tri_attn.h.  Z_rows is the slab of problem rows row0.. of an
+    # N x N problem ([nrows][N][c_z]); the starting-node formula applies (an
+    # ending-node block is the starting-node block of the transposed tensor).
+    def bias_ld(self, N: int) -> int:
+        return int(lib().tri_attn_bias_ld(int(N)))
+
+    def rows_bias(self, Z_rows: torch.Tensor, N: int, row0: int, mask=None,
+                  bias_rows: torch.Tensor | None = None, stream=None, flags: int = 0):
+        """The slab's logit-bias rows, [H][nrows][ld] bf16."""
+        assert Z_rows.is_cuda and Z_rows.dtype == self.dtype and Z_rows.is_contiguous()
+        nrows = Z_rows.shape[0]
+        if bias_rows is None:
+            bias_rows = torch.empty(4, nrows, self.bias_ld(N), dtype=torch.bfloat16,
+                                    device=Z_rows.device)
+        if mask is not None:
+            mask = mask.to(device=Z_rows.device, dtype=torch.uint8).contiguous()
+        rc = lib().tri_attn_rows_bias(self.handle, _ptr(Z_rows), int(N), int(row0), nrows,
+                                      _ptr(mask), _ptr(bias_rows), _stream_handle(stream), flags)
+        if rc != TRI_ATTN_OK:
+            raise TriAttnError(rc, "tri_attn_rows_bias")
+        return bias_rows
+
+    def rows_forward(self, Z_rows: torch.Tensor, N: int, row0: int, bias_all: torch.Tensor,
+                     mask=None, out: torch.Tensor | None = None, stream=None, flags: int = 0):
+        """The starting-node block on the slab, given the whole [H][N][ld] bias."""
+        assert Z_rows.is_cuda and Z_rows.dtype == self.dtype and Z_rows.is_contiguous()
+        assert bias_all.is_cuda and bias_all.is_contiguous()
+        if out is None:
+            out = torch.empty_like(Z_rows)
+        if mask is not None:
+            mask = mask.to(device=Z_rows.device, dtype=torch.uint8).contiguous()
+        rc = lib().tri_attn_rows_forward(self.handle, _ptr(Z_rows), int(N), int(row0),
+                                         Z_rows.shape[0], _ptr(mask), _ptr(bias_all), _ptr(out),
+                                         _stream_handle(stream), flags)
+        if rc != TRI_ATTN_OK:
+            raise TriAttnError(rc, "tri_attn_rows_forward")
         return out
 
     def status(self, stream=None) -> int:

@@ -63,6 +63,9 @@ struct ProjArgs {
   float eps, q_scale;
   __nv_bfloat16 *Q, *K, *V, *G, *bias;
   int ld_bias;
+  // Z holds problem rows z_row0.. (a row slab; 0 for the whole tensor), and the
+  // bias buffer holds, per head, bias_rows problem rows starting at bias_row0
+  int z_row0, bias_row0, bias_rows;
   int* status;
 };
 
@@ -79,6 +82,7 @@ struct GateArgs {
   const float* b_o;
   __nv_bfloat16* out;
   int N, orient, row0, rows;
+  int z_row0;  // Z and out hold problem rows z_row0.. (a row slab; 0 for the whole tensor)
   int* status;
 };
 

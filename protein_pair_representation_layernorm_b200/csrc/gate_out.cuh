@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i = a.row0 + r;
     if (a.orient == 0) {
       c1 = j0;
-      c2 = i;
+      c2 = i - a.z_row0;
     } else {
       c1 = i;
       c2 = j0;

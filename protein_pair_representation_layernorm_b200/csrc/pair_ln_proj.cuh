@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = static_cast<int>(t / jtiles);
     const int j0 = static_cast<int>(t % jtiles) * kTileM;
     const int i = a.row0 + r;
-    const int c1 = a.orient == 0 ? j0 : i, c2 = a.orient == 0 ? i : j0;
+    const int c1 = a.orient == 0 ? j0 : i, c2 = a.orient == 0 ? i - a.z_row0 : j0;
     mbar_arrive_expect_tx(&z_full[grp], kATileBytes);
     tma_load_3d(sA, &map_z, &z_full[grp], 0, c1, c2);
     tma_load_3d(sA + kAAtomBytes, &map_z, &z_full[grp], 64, c1, c2);
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (j < a.ld_bias) {
 #pragma unroll
         for (int h = 0; h < kHeads; ++h)
-          a.bias[(static_cast<long long>(h) * a.N + i) * a.ld_bias + j] =
+          a.bias[(static_cast<long long>(h) * a.bias_rows + (i - a.bias_row0)) * a.ld_bias + j] =
               __float2bfloat16_rn(key_valid ? bacc[h].x + bacc[h].y : kMaskedLogit);
       }
     }

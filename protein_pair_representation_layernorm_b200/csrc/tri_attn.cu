@@ -159,10 +159,18 @@ int upload(const std::vector<T>& v, void** dst) {
   return TRI_ATTN_OK;
 }
 
-bool attrs_set = false;
+// cudaFuncSetAttribute applies to the current device only: record per device
+// that the kernels' shared-memory limits were raised there.
+constexpr int kMaxAttrDevices = 64;
+std::mutex g_attrs_mutex;
+bool g_attrs_set[kMaxAttrDevices] = {};
 
 int set_kernel_attrs() {
-  if (attrs_set) return TRI_ATTN_OK;
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxAttrDevices) return TRI_ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_attrs_mutex);
+  if (g_attrs_set[dev]) return TRI_ATTN_OK;
   CUDA_TRY(cudaFuncSetAttribute(tri::plp::pair_ln_proj, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 tri::plp::kSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(tri::attn::tri_attn_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -175,7 +183,7 @@ int set_kernel_attrs() {
       TA_LOG("tri_attn_fwd: regs %d, max threads %d, static smem %zu, local %zu", fa.numRegs,
              fa.maxThreadsPerBlock, fa.sharedSizeBytes, fa.localSizeBytes);
   }
-  attrs_set = true;
+  g_attrs_set[dev] = true;
   return TRI_ATTN_OK;
 }
 
@@ -293,24 +301,36 @@ bool ranges_overlap(const void* a, const void* b, size_t bytes) {
   return x < y + bytes && y < x + bytes;
 }
 
+// A row slab of a starting-node block (bf16): Z and out hold problem rows
+// row0 .. row0+nrows-1.  Phase 0 writes the slab's logit-bias rows to bias_io
+// ([H][nrows][ld]); phase 1 runs the block on the slab with bias_io as the
+// whole problem's bias ([H][N][ld]).
+struct RowSlab {
+  int row0, nrows, phase;
+  void* bias_io;
+};
+
 int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, int orient,
-                 void* out, cudaStream_t st, unsigned flags) {
+                 void* out, cudaStream_t st, unsigned flags, const RowSlab* slab = nullptr) {
   const tri_attn_dtype dt = h->dtype;
   const bool timed = (flags & TRI_ATTN_FLAG_TIME_KERNELS) != 0;
   const int ld = ld_bias_for(N);
+  const int rbeg = slab ? slab->row0 : 0;           // problem rows of this call
+  const int rend = slab ? slab->row0 + slab->nrows : N;
+  const int zrows = rend - rbeg;                     // rows Z and out hold
 
   // rows per chunk under the workspace limit
-  const size_t full = layout_for(dt, N, N).total;
-  int rows = N;
+  const size_t full = layout_for(dt, N, zrows).total;
+  int rows = zrows;
   if (full > h->ws_limit) {
     const size_t fixed = bias_bytes(dt, N) + 6 * 256;
     if (h->ws_limit <= fixed) return TRI_ATTN_ERR_OOM;
     size_t fit = (h->ws_limit - fixed) / row_bytes(dt, N);
     fit = fit / tri::attn::kRows * tri::attn::kRows;
     if (fit < static_cast<size_t>(tri::attn::kRows)) return TRI_ATTN_ERR_OOM;
-    rows = static_cast<int>(std::min<size_t>(fit, static_cast<size_t>(N)));
+    rows = static_cast<int>(std::min<size_t>(fit, static_cast<size_t>(zrows)));
   }
-  const bool chunked = rows < N;
+  const bool chunked = rows < zrows;
   const Layout L = layout_for(dt, N, rows);
   int rc = ensure_workspace(h, L.total);
   if (rc != TRI_ATTN_OK) return rc;
@@ -320,7 +340,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
   h->v = ws + L.v;
   h->g = ws + L.g;
   h->o = ws + L.o;
-  h->bias = ws + L.bias;
+  h->bias = (slab && slab->phase == 1) ? slab->bias_io : static_cast<void*>(ws + L.bias);
   h->ld_bias = ld;
   TA_LOG("forward N=%d orient=%d dtype=%d rows/chunk=%d ws=%zu", N, orient, static_cast<int>(dt),
          rows, L.total);
@@ -432,8 +452,11 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
     a.K = static_cast<bf16*>(h->k);
     a.V = static_cast<bf16*>(h->v);
     a.G = static_cast<bf16*>(h->g);
-    a.bias = static_cast<bf16*>(h->bias);
+    a.bias = static_cast<bf16*>(slab && slab->phase == 0 ? slab->bias_io : h->bias);
     a.ld_bias = ld;
+    a.z_row0 = rbeg;
+    a.bias_row0 = slab && slab->phase == 0 ? rbeg : 0;
+    a.bias_rows = slab && slab->phase == 0 ? zrows : N;
     a.status = h->status;
     const long long ntiles = static_cast<long long>(nrows) * jtiles;
     const unsigned grid = static_cast<unsigned>(
@@ -442,7 +465,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
     // the swapped view, along the rows of Z (ending node)
     CUtensorMap mz;
     const uint32_t zb1 = orient == 0 ? 128u : 1u, zb2 = orient == 0 ? 1u : 128u;
-    if (!make_map_3d(&mz, Zb, kCz, N, N, kCz * 2, static_cast<uint64_t>(N) * kCz * 2, 64, zb1,
+    if (!make_map_3d(&mz, Zb, kCz, N, zrows, kCz * 2, static_cast<uint64_t>(N) * kCz * 2, 64, zb1,
                      CU_TENSOR_MAP_SWIZZLE_128B, zb2))
       return cudaErrorInvalidValue;
     // q, k, v, g outputs ([rows][H][N][d] bf16): 32 x 32 boxes, 64 B swizzle (the
@@ -459,10 +482,16 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
         mz, mo[0], mo[1], mo[2], mo[3], a);
     return cudaGetLastError();
   };
-  if (chunked) CUDA_TRY(proj(0, N, 0, 1));
-  for (int r0 = 0; r0 < N; r0 += rows) {
-    const int nr = std::min(rows, N - r0);
-    CUDA_TRY(proj(r0, nr, 1, chunked ? 0 : 1));
+  if (slab && slab->phase == 0) {  // the slab's bias rows only
+    CUDA_TRY(proj(rbeg, zrows, 0, 1));
+    CUDA_TRY(cudaGetLastError());
+    return TRI_ATTN_OK;
+  }
+  const bool own_bias = slab == nullptr;
+  if (chunked && own_bias) CUDA_TRY(proj(0, N, 0, 1));
+  for (int r0 = rbeg; r0 < rend; r0 += rows) {
+    const int nr = std::min(rows, rend - r0);
+    CUDA_TRY(proj(r0, nr, 1, (chunked || !own_bias) ? 0 : 1));
     {
       CUtensorMap mq, mk, mv, mb;
       const uint64_t rh = static_cast<uint64_t>(nr) * kHeads;
@@ -500,9 +529,10 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
                       static_cast<uint64_t>(N) * kD * 2, kD, 128, CU_TENSOR_MAP_SWIZZLE_64B) &&
           make_map_3d(&mg, h->g, kD, N, static_cast<uint64_t>(nr) * kHeads, kD * 2,
                       static_cast<uint64_t>(N) * kD * 2, kD, 128, CU_TENSOR_MAP_SWIZZLE_64B) &&
-          make_map_3d(&mz, Zb, kCz, N, N, kCz * 2, rowb, 64, zb1, CU_TENSOR_MAP_SWIZZLE_128B, zb2) &&
-          make_map_3d(&mout, outb, kCz, N, N, kCz * 2, rowb, 64, zb1, CU_TENSOR_MAP_SWIZZLE_128B,
-                      zb2);
+          make_map_3d(&mz, Zb, kCz, N, zrows, kCz * 2, rowb, 64, zb1, CU_TENSOR_MAP_SWIZZLE_128B,
+                      zb2) &&
+          make_map_3d(&mout, outb, kCz, N, zrows, kCz * 2, rowb, 64, zb1,
+                      CU_TENSOR_MAP_SWIZZLE_128B, zb2);
       if (!okm) return TRI_ATTN_ERR_CUDA;
       tri::GateArgs a{};
       a.Z = Zb;
@@ -515,6 +545,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
       a.orient = orient;
       a.row0 = r0;
       a.rows = nr;
+      a.z_row0 = rbeg;
       a.status = h->status;
       const long long ntiles = static_cast<long long>(nr) * jtiles;
       const unsigned grid = static_cast<unsigned>(std::min<long long>(ntiles, h->num_sms));
@@ -524,7 +555,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
       CUDA_TRY(cudaGetLastError());
     }
   }
-  h->rows_last = N - (N - 1) / rows * rows;
+  h->rows_last = zrows - (zrows - 1) / rows * rows;
   CUDA_TRY(cudaGetLastError());
   return TRI_ATTN_OK;
 }
@@ -674,6 +705,60 @@ int tri_attn_forward(tri_attn_handle* h, const void* Z, int N, const uint8_t* ma
     return read_status(h, st);
   }
   return TRI_ATTN_OK;
+}
+
+namespace {
+// Shared checks of the two row-slab entry points.
+int check_rows_args(tri_attn_handle* h, const void* Z_rows, int N, int row0, int nrows,
+                    const void* bias, const void* out_rows) {
+  if (!h || !Z_rows || !bias || N < 1 || row0 < 0 || nrows < 1 || row0 > N - nrows)
+    return TRI_ATTN_ERR_INVALID_ARG;
+  if (h->dtype != TRI_ATTN_BF16) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (N > 46340) return TRI_ATTN_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(Z_rows) & 15) || (reinterpret_cast<uintptr_t>(bias) & 15) ||
+      (out_rows && (reinterpret_cast<uintptr_t>(out_rows) & 15)))
+    return TRI_ATTN_ERR_INVALID_ARG;
+  return TRI_ATTN_OK;
+}
+
+int finish_call(tri_attn_handle* h, cudaStream_t st, unsigned flags) {
+  if (flags & TRI_ATTN_FLAG_SYNC) {
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+    return read_status(h, st);
+  }
+  return TRI_ATTN_OK;
+}
+}  // namespace
+
+int tri_attn_bias_ld(int N) { return N < 1 ? 0 : ld_bias_for(N); }
+
+int tri_attn_rows_bias(tri_attn_handle* h, const void* Z_rows, int N, int row0, int nrows,
+                       const uint8_t* mask, void* bias_rows, void* stream, unsigned flags) {
+  int rc = check_rows_args(h, Z_rows, N, row0, nrows, bias_rows, nullptr);
+  if (rc != TRI_ATTN_OK) return rc;
+  if (cudaSetDevice(h->device) != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const RowSlab slab{row0, nrows, 0, bias_rows};
+  rc = forward_impl(h, Z_rows, N, mask, TRI_ATTN_STARTING, nullptr, st, flags, &slab);
+  if (rc != TRI_ATTN_OK) return rc;
+  return finish_call(h, st, flags);
+}
+
+int tri_attn_rows_forward(tri_attn_handle* h, const void* Z_rows, int N, int row0, int nrows,
+                          const uint8_t* mask, const void* bias_all, void* out_rows,
+                          void* stream, unsigned flags) {
+  int rc = check_rows_args(h, Z_rows, N, row0, nrows, bias_all, out_rows);
+  if (rc != TRI_ATTN_OK) return rc;
+  if (!out_rows) return TRI_ATTN_ERR_INVALID_ARG;
+  const size_t bytes = static_cast<size_t>(nrows) * N * kCz * 2;
+  if (Z_rows != out_rows && ranges_overlap(Z_rows, out_rows, bytes)) return TRI_ATTN_ERR_ALIAS;
+  if (cudaSetDevice(h->device) != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const RowSlab slab{row0, nrows, 1, const_cast<void*>(bias_all)};
+  rc = forward_impl(h, Z_rows, N, mask, TRI_ATTN_STARTING, out_rows, st, flags, &slab);
+  if (rc != TRI_ATTN_OK) return rc;
+  return finish_call(h, st, flags);
 }
 
 int tri_attn_forward_host(tri_attn_handle* h, const void* Z_host, int N, const uint8_t* mask_host,
