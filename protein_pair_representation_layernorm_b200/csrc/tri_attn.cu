@@ -152,6 +152,7 @@ int copy_to_host_f32(const void* dev, size_t n, tri_attn_dtype dt, std::vector<f
   return TRI_ATTN_OK;
 }
 
+// *dst is set whenever the allocation succeeded, also if the copy then fails.
 template <class T>
 int upload(const std::vector<T>& v, void** dst) {
   CUDA_TRY(cudaMalloc(dst, v.size() * sizeof(T)));
@@ -668,17 +669,18 @@ int tri_attn_create(const tri_attn_params* p, tri_attn_handle** out) {
     if ((rc = upload(w512, &h->w_qkvg))) return fail(rc);
     if ((rc = upload(wo, &h->w_o))) return fail(rc);
   }
-  void* tmp = nullptr;
-  if ((rc = upload(wb, &tmp))) return fail(rc);
-  h->w_b = static_cast<float*>(tmp);
-  if ((rc = upload(gamma, &tmp))) return fail(rc);
-  h->gamma = static_cast<float*>(tmp);
-  if ((rc = upload(beta, &tmp))) return fail(rc);
-  h->beta = static_cast<float*>(tmp);
-  if ((rc = upload(bg, &tmp))) return fail(rc);
-  h->b_g = static_cast<float*>(tmp);
-  if ((rc = upload(bo, &tmp))) return fail(rc);
-  h->b_o = static_cast<float*>(tmp);
+  // the handle owns each buffer as soon as it is allocated, so a failure part
+  // way through is cleaned up by tri_attn_destroy
+  auto upload_to = [&](const std::vector<float>& v, float** field) {
+    void* t = nullptr;
+    const int r = upload(v, &t);
+    *field = static_cast<float*>(t);
+    return r;
+  };
+  if ((rc = upload_to(wb, &h->w_b)) || (rc = upload_to(gamma, &h->gamma)) ||
+      (rc = upload_to(beta, &h->beta)) || (rc = upload_to(bg, &h->b_g)) ||
+      (rc = upload_to(bo, &h->b_o)))
+    return fail(rc);
   if (cudaMalloc(&h->status, sizeof(int)) != cudaSuccess) return fail(TRI_ATTN_ERR_OOM);
   if (cudaMemset(h->status, 0, sizeof(int)) != cudaSuccess) return fail(TRI_ATTN_ERR_CUDA);
   *out = h;
