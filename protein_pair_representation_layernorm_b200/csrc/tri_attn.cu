@@ -20,6 +20,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <functional>
 #include <mutex>
 #include <new>
 #include <vector>
@@ -221,6 +222,10 @@ struct tri_attn_handle {
   size_t stage_bytes = 0;
   uint8_t* stage_mask = nullptr;
   size_t stage_mask_bytes = 0;
+  // forward_host: the stream its read-back copies run on, and the event that
+  // orders each copy after the chunk that produced it
+  cudaStream_t copy_st = nullptr;
+  cudaEvent_t chunk_ev = nullptr;
   // kernel timing
   std::vector<EventPair> ev[3];
   int ev_used[3] = {0, 0, 0};
@@ -311,8 +316,17 @@ struct RowSlab {
   void* bias_io;
 };
 
+// Optional per-chunk hook: at most max_rows problem rows per chunk (0 = no
+// cap), and after(r0, nr) called once each chunk's output rows r0..r0+nr-1
+// are enqueued (after its gate_out launch, on the call's stream).
+struct ChunkHook {
+  int max_rows;
+  std::function<int(int, int)> after;
+};
+
 int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, int orient,
-                 void* out, cudaStream_t st, unsigned flags, const RowSlab* slab = nullptr) {
+                 void* out, cudaStream_t st, unsigned flags, const RowSlab* slab = nullptr,
+                 const ChunkHook* hook = nullptr) {
   const tri_attn_dtype dt = h->dtype;
   const bool timed = (flags & TRI_ATTN_FLAG_TIME_KERNELS) != 0;
   const int ld = ld_bias_for(N);
@@ -331,6 +345,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
     if (fit < static_cast<size_t>(tri::attn::kRows)) return TRI_ATTN_ERR_OOM;
     rows = static_cast<int>(std::min<size_t>(fit, static_cast<size_t>(zrows)));
   }
+  if (hook && hook->max_rows > 0 && hook->max_rows < rows) rows = hook->max_rows;
   const bool chunked = rows < zrows;
   const Layout L = layout_for(dt, N, rows);
   int rc = ensure_workspace(h, L.total);
@@ -419,6 +434,11 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
         tri::f32::gate_out_kernel<<<static_cast<unsigned>((pairs + tri::f32::kProjThreads - 1) /
                                                           tri::f32::kProjThreads),
                                     tri::f32::kProjThreads, 0, st>>>(a);
+      }
+      if (hook && hook->after) {
+        CUDA_TRY(cudaGetLastError());
+        const int hrc = hook->after(r0, nr);
+        if (hrc != TRI_ATTN_OK) return hrc;
       }
     }
     h->rows_last = std::min(rows, N - (N - 1) / rows * rows);
@@ -554,6 +574,10 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
       tri::gout::gate_out<<<grid, tri::gout::kThreads, tri::gout::kSmemBytes, st>>>(mo, mg, mz,
                                                                                    mout, a);
       CUDA_TRY(cudaGetLastError());
+    }
+    if (hook && hook->after) {
+      const int hrc = hook->after(r0, nr);
+      if (hrc != TRI_ATTN_OK) return hrc;
     }
   }
   h->rows_last = zrows - (zrows - 1) / rows * rows;
@@ -796,12 +820,47 @@ int tri_attn_forward_host(tri_attn_handle* h, const void* Z_host, int N, const u
     dmask = h->stage_mask;
   }
   CUDA_TRY(cudaMemcpyAsync(h->stage, Z_host, bytes, cudaMemcpyHostToDevice, st));
-  for (int t = 0; t < n_orientations; ++t) {
+  if (n_orientations == 0) {
+    CUDA_TRY(cudaMemcpyAsync(out_host, h->stage, bytes, cudaMemcpyDeviceToHost, st));
+    CUDA_TRY(cudaStreamSynchronize(st));
+    return read_status(h, st);
+  }
+  for (int t = 0; t + 1 < n_orientations; ++t) {
     int rc = forward_impl(h, h->stage, N, dmask, orientations[t], h->stage, st,
                           flags & ~TRI_ATTN_FLAG_SYNC);
     if (rc != TRI_ATTN_OK) return rc;
   }
-  CUDA_TRY(cudaMemcpyAsync(out_host, h->stage, bytes, cudaMemcpyDeviceToHost, st));
+  // The last block runs in row chunks (about 8), and each chunk's output goes
+  // back to the host on a second stream as soon as its gate_out has run, while
+  // the later chunks compute: a chunk's output region (rows of Z for the
+  // starting node, columns for the ending node) is final once written, and no
+  // later chunk reads or writes it.
+  if (!h->copy_st) CUDA_TRY(cudaStreamCreateWithFlags(&h->copy_st, cudaStreamNonBlocking));
+  if (!h->chunk_ev) CUDA_TRY(cudaEventCreateWithFlags(&h->chunk_ev, cudaEventDisableTiming));
+  const int last = orientations[n_orientations - 1];
+  const size_t es = esize(h->dtype), pair_b = kCz * es, row_b = static_cast<size_t>(N) * pair_b;
+  ChunkHook hook;
+  hook.max_rows = std::max(tri::attn::kRows,
+                           ((N + 7) / 8 + tri::attn::kRows - 1) / tri::attn::kRows * tri::attn::kRows);
+  hook.after = [&](int r0, int nr) -> int {
+    CUDA_TRY(cudaEventRecord(h->chunk_ev, st));
+    CUDA_TRY(cudaStreamWaitEvent(h->copy_st, h->chunk_ev, 0));
+    char* dst = static_cast<char*>(out_host);
+    const char* src = static_cast<const char*>(h->stage);
+    if (last == TRI_ATTN_STARTING) {
+      CUDA_TRY(cudaMemcpyAsync(dst + r0 * row_b, src + r0 * row_b, nr * row_b,
+                               cudaMemcpyDeviceToHost, h->copy_st));
+    } else {  // columns r0 .. r0+nr-1 of every row
+      CUDA_TRY(cudaMemcpy2DAsync(dst + r0 * pair_b, row_b, src + r0 * pair_b, row_b, nr * pair_b,
+                                 static_cast<size_t>(N), cudaMemcpyDeviceToHost, h->copy_st));
+    }
+    return TRI_ATTN_OK;
+  };
+  int rc = forward_impl(h, h->stage, N, dmask, last, h->stage, st, flags & ~TRI_ATTN_FLAG_SYNC,
+                        nullptr, &hook);
+  const cudaError_t e_copy = cudaStreamSynchronize(h->copy_st);
+  if (rc != TRI_ATTN_OK) return rc;
+  if (e_copy != cudaSuccess) return TRI_ATTN_ERR_CUDA;
   CUDA_TRY(cudaStreamSynchronize(st));
   return read_status(h, st);
 }
@@ -861,6 +920,8 @@ int tri_attn_destroy(tri_attn_handle* h) {
       if (p.a) cudaEventDestroy(p.a);
       if (p.b) cudaEventDestroy(p.b);
     }
+  if (h->chunk_ev) cudaEventDestroy(h->chunk_ev);
+  if (h->copy_st) cudaStreamDestroy(h->copy_st);
   delete h;
   return TRI_ATTN_OK;
 }

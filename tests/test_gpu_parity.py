@@ -150,14 +150,24 @@ def test_sequence_starting_then_ending():
     assert_within(st, "bf16", "start then end")
 
 
-def test_host_buffer_entry_point():
-    inp = workloads.make_inputs(120, "bf16", 45, "random:0.1")
+# The last block of a host-buffer call runs in ~8 row chunks whose outputs are
+# read back while later chunks compute (rows of Z when the starting node comes
+# last, strided columns when the ending node does): the result must equal the
+# device path bit for bit.
+@pytest.mark.parametrize("N,dtype,orients", [(120, "bf16", [0, 1]), (97, "bf16", [1, 0]),
+                                             (130, "bf16", [1]), (64, "bf16", [0]),
+                                             (70, "f32", [0, 1]), (33, "bf16", [])])
+def test_host_buffer_entry_point(N, dtype, orients):
+    inp = workloads.make_inputs(N, dtype, 45 + N, "random:0.1")
     blk = block_for(inp)
     z_host = inp.Z.clone().pin_memory()
-    got = blk.forward_host(z_host, [0, 1], inp.mask)
-    out1 = blk.forward(inp.Z.cuda(), 0, inp.mask.cuda())
-    out2 = blk.forward(out1, 1, inp.mask.cuda(), flags=binding.TRI_ATTN_FLAG_SYNC)
-    assert torch.equal(got.view(torch.int16), out2.cpu().view(torch.int16))
+    got = blk.forward_host(z_host, orients, inp.mask)
+    want = inp.Z.cuda()
+    for o in orients:
+        want = blk.forward(want, o, inp.mask.cuda(), flags=binding.TRI_ATTN_FLAG_SYNC)
+    bits = torch.int16 if dtype == "bf16" else torch.int32
+    assert torch.equal(got.view(bits), want.cpu().view(bits))
+    assert torch.equal(z_host, inp.Z)  # the input buffer is left alone
 
 
 def test_kernel_times_reported():
