@@ -109,9 +109,11 @@ int tri_attn_forward(tri_attn_handle *h, const void *Z, int N, const uint8_t *ma
  * output of the previous one (in place in a device staging buffer owned by
  * the handle), and copies the final result back to out_host.  Synchronous:
  * returns after out_host is written.  Z_host and out_host may be the same
- * buffer; pinned host memory gives full PCIe bandwidth.  The last block runs
- * in row chunks whose results are copied back while later chunks compute, so
- * most of the device-to-host copy overlaps the computation. */
+ * buffer; pinned host memory gives full PCIe bandwidth.  Z is copied in
+ * pieces that the first block's projection consumes as they arrive, and the
+ * last block runs in row chunks whose results are copied back while later
+ * chunks compute, so the copies overlap the computation where the block's
+ * data dependencies allow. */
 int tri_attn_forward_host(tri_attn_handle *h, const void *Z_host, int N,
                           const uint8_t *mask_host, const int *orientations,
                           int n_orientations, void *out_host, void *stream,

@@ -226,6 +226,8 @@ struct tri_attn_handle {
   // orders each copy after the chunk that produced it
   cudaStream_t copy_st = nullptr;
   cudaEvent_t chunk_ev = nullptr;
+  static constexpr int kInRanges = 8;  // input copies of forward_host, one event each
+  cudaEvent_t in_ev[kInRanges] = {};
   // kernel timing
   std::vector<EventPair> ev[3];
   int ev_used[3] = {0, 0, 0};
@@ -320,8 +322,13 @@ struct RowSlab {
 // cap), and after(r0, nr) called once each chunk's output rows r0..r0+nr-1
 // are enqueued (after its gate_out launch, on the call's stream).
 struct ChunkHook {
-  int max_rows;
+  int max_rows = 0;
   std::function<int(int, int)> after;
+  // bf16, unchunked calls only: the projection runs in launches of
+  // proj_split_rows rows, each preceded by before_proj(r0, nr) (which may make
+  // the stream wait for those rows' input)
+  int proj_split_rows = 0;
+  std::function<int(int, int)> before_proj;
 };
 
 int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, int orient,
@@ -452,7 +459,8 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
   const bf16* Zb = static_cast<const bf16*>(Z);
   bf16* outb = static_cast<bf16*>(out);
   const int jtiles = (N + 127) / 128;
-  auto proj = [&](int row0, int nrows, int wq, int wb) {
+  auto proj = [&](int row0, int nrows, int wq, int wb, int out_off = 0) {
+    const size_t off = static_cast<size_t>(out_off) * kHeads * N * kD;  // rows into Q/K/V/G
     tri::ProjArgs a{};
     a.Z = Zb;
     a.mask = mask;
@@ -469,10 +477,10 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
     a.b_g = h->b_g;
     a.eps = h->eps;
     a.q_scale = h->q_scale;
-    a.Q = static_cast<bf16*>(h->q);
-    a.K = static_cast<bf16*>(h->k);
-    a.V = static_cast<bf16*>(h->v);
-    a.G = static_cast<bf16*>(h->g);
+    a.Q = static_cast<bf16*>(h->q) + off;
+    a.K = static_cast<bf16*>(h->k) + off;
+    a.V = static_cast<bf16*>(h->v) + off;
+    a.G = static_cast<bf16*>(h->g) + off;
     a.bias = static_cast<bf16*>(slab && slab->phase == 0 ? slab->bias_io : h->bias);
     a.ld_bias = ld;
     a.z_row0 = rbeg;
@@ -492,7 +500,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
     // q, k, v, g outputs ([rows][H][N][d] bf16): 32 x 32 boxes, 64 B swizzle (the
     // kernel's per-warp staging layout); a bias-only pass never stores through them
     CUtensorMap mo[4];
-    void* outs[4] = {h->q, h->k, h->v, h->g};
+    void* outs[4] = {a.Q, a.K, a.V, a.G};
     const uint64_t rh = static_cast<uint64_t>(wq ? nrows : 1) * kHeads;
     for (int m = 0; m < 4; ++m)
       if (!make_map_3d(&mo[m], outs[m], kD, N, rh, kD * 2, static_cast<uint64_t>(N) * kD * 2, kD,
@@ -512,7 +520,16 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
   if (chunked && own_bias) CUDA_TRY(proj(0, N, 0, 1));
   for (int r0 = rbeg; r0 < rend; r0 += rows) {
     const int nr = std::min(rows, rend - r0);
-    CUDA_TRY(proj(r0, nr, 1, (chunked || !own_bias) ? 0 : 1));
+    if (!chunked && own_bias && hook && hook->before_proj && hook->proj_split_rows > 0) {
+      for (int p0 = r0; p0 < r0 + nr; p0 += hook->proj_split_rows) {
+        const int pn = std::min(hook->proj_split_rows, r0 + nr - p0);
+        const int hrc = hook->before_proj(p0, pn);
+        if (hrc != TRI_ATTN_OK) return hrc;
+        CUDA_TRY(proj(p0, pn, 1, 1, p0 - r0));
+      }
+    } else {
+      CUDA_TRY(proj(r0, nr, 1, (chunked || !own_bias) ? 0 : 1));
+    }
     {
       CUtensorMap mq, mk, mv, mb;
       const uint64_t rh = static_cast<uint64_t>(nr) * kHeads;
@@ -819,26 +836,68 @@ int tri_attn_forward_host(tri_attn_handle* h, const void* Z_host, int N, const u
     CUDA_TRY(cudaMemcpyAsync(h->stage_mask, mask_host, N, cudaMemcpyHostToDevice, st));
     dmask = h->stage_mask;
   }
-  CUDA_TRY(cudaMemcpyAsync(h->stage, Z_host, bytes, cudaMemcpyHostToDevice, st));
+  if (!h->copy_st) CUDA_TRY(cudaStreamCreateWithFlags(&h->copy_st, cudaStreamNonBlocking));
+  if (!h->chunk_ev) CUDA_TRY(cudaEventCreateWithFlags(&h->chunk_ev, cudaEventDisableTiming));
+  const size_t es = esize(h->dtype), pair_b = kCz * es, row_b = static_cast<size_t>(N) * pair_b;
+  // With two or more blocks and an unchunked bf16 first block, Z goes to the
+  // device in kInRanges pieces on the copy stream (rows of Z when the first
+  // block is a starting node, columns when it is an ending node), and the
+  // first block's projection of each piece starts as soon as that piece has
+  // arrived; everything after the projection needs the whole bias and waits
+  // for all pieces.
+  const bool pipelined_in = n_orientations >= 2 && h->dtype == TRI_ATTN_BF16 &&
+                            layout_for(h->dtype, N, N).total <= h->ws_limit &&
+                            N >= tri_attn_handle::kInRanges;
+  const int in_split = (N + tri_attn_handle::kInRanges - 1) / tri_attn_handle::kInRanges;
+  if (pipelined_in) {
+    const int first = orientations[0];
+    for (int c = 0; c < tri_attn_handle::kInRanges; ++c) {
+      if (!h->in_ev[c]) CUDA_TRY(cudaEventCreateWithFlags(&h->in_ev[c], cudaEventDisableTiming));
+      const int r0 = c * in_split, nr = std::min(in_split, N - r0);
+      if (nr <= 0) continue;
+      char* dst = static_cast<char*>(h->stage);
+      const char* src = static_cast<const char*>(Z_host);
+      if (first == TRI_ATTN_STARTING) {
+        CUDA_TRY(cudaMemcpyAsync(dst + r0 * row_b, src + r0 * row_b, nr * row_b,
+                                 cudaMemcpyHostToDevice, h->copy_st));
+      } else {  // columns r0 .. r0+nr-1 of every row
+        CUDA_TRY(cudaMemcpy2DAsync(dst + r0 * pair_b, row_b, src + r0 * pair_b, row_b,
+                                   nr * pair_b, static_cast<size_t>(N), cudaMemcpyHostToDevice,
+                                   h->copy_st));
+      }
+      CUDA_TRY(cudaEventRecord(h->in_ev[c], h->copy_st));
+    }
+  } else {
+    CUDA_TRY(cudaMemcpyAsync(h->stage, Z_host, bytes, cudaMemcpyHostToDevice, st));
+  }
   if (n_orientations == 0) {
     CUDA_TRY(cudaMemcpyAsync(out_host, h->stage, bytes, cudaMemcpyDeviceToHost, st));
     CUDA_TRY(cudaStreamSynchronize(st));
     return read_status(h, st);
   }
   for (int t = 0; t + 1 < n_orientations; ++t) {
+    ChunkHook in_hook;
+    if (t == 0 && pipelined_in) {
+      in_hook.proj_split_rows = in_split;
+      in_hook.before_proj = [&](int r0, int) -> int {
+        CUDA_TRY(cudaStreamWaitEvent(st, h->in_ev[r0 / in_split], 0));
+        return TRI_ATTN_OK;
+      };
+    }
     int rc = forward_impl(h, h->stage, N, dmask, orientations[t], h->stage, st,
-                          flags & ~TRI_ATTN_FLAG_SYNC);
-    if (rc != TRI_ATTN_OK) return rc;
+                          flags & ~TRI_ATTN_FLAG_SYNC, nullptr,
+                          (t == 0 && pipelined_in) ? &in_hook : nullptr);
+    if (rc != TRI_ATTN_OK) {
+      cudaStreamSynchronize(h->copy_st);
+      return rc;
+    }
   }
   // The last block runs in row chunks (about 8), and each chunk's output goes
   // back to the host on a second stream as soon as its gate_out has run, while
   // the later chunks compute: a chunk's output region (rows of Z for the
   // starting node, columns for the ending node) is final once written, and no
   // later chunk reads or writes it.
-  if (!h->copy_st) CUDA_TRY(cudaStreamCreateWithFlags(&h->copy_st, cudaStreamNonBlocking));
-  if (!h->chunk_ev) CUDA_TRY(cudaEventCreateWithFlags(&h->chunk_ev, cudaEventDisableTiming));
   const int last = orientations[n_orientations - 1];
-  const size_t es = esize(h->dtype), pair_b = kCz * es, row_b = static_cast<size_t>(N) * pair_b;
   ChunkHook hook;
   hook.max_rows = std::max(tri::attn::kRows,
                            ((N + 7) / 8 + tri::attn::kRows - 1) / tri::attn::kRows * tri::attn::kRows);
@@ -921,6 +980,8 @@ int tri_attn_destroy(tri_attn_handle* h) {
       if (p.b) cudaEventDestroy(p.b);
     }
   if (h->chunk_ev) cudaEventDestroy(h->chunk_ev);
+  for (cudaEvent_t e : h->in_ev)
+    if (e) cudaEventDestroy(e);
   if (h->copy_st) cudaStreamDestroy(h->copy_st);
   delete h;
   return TRI_ATTN_OK;
