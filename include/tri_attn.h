@@ -34,6 +34,10 @@
  * thread.  Results are deterministic (no floating-point atomics).
  * There is no CPU fallback: without a usable sm_100 device every call that
  * needs one returns TRI_ATTN_ERR_NO_DEVICE.
+ *
+ * Diagnostics: with the environment variable TRIATTN_LOG=1 the library prints
+ * to stderr why a call failed (the CUDA call and its error, a rejected size)
+ * and, per forward, the row chunking and workspace size it chose.
  */
 #ifndef TRI_ATTN_H
 #define TRI_ATTN_H
