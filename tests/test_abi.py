@@ -90,3 +90,16 @@ def test_product_path_never_touches_the_oracle():
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
                 assert "liboracle" not in text, f
                 assert "oracle.c" not in text, f
+
+
+def test_row_slab_calls_reject_bad_arguments_without_device():
+    L = binding.lib()
+    assert L.tri_attn_bias_ld(0) == 0
+    assert L.tri_attn_bias_ld(1) == 64 and L.tri_attn_bias_ld(64) == 64
+    assert L.tri_attn_bias_ld(65) == 128 and L.tri_attn_bias_ld(1536) == 1536
+    buf = ctypes.c_void_p(0x10000)
+    # no handle: rejected before anything else
+    assert L.tri_attn_rows_bias(None, buf, 16, 0, 16, None, buf, None, 0) == \
+        binding.TRI_ATTN_ERR_INVALID_ARG
+    assert L.tri_attn_rows_forward(None, buf, 16, 0, 16, None, buf, buf, None, 0) == \
+        binding.TRI_ATTN_ERR_INVALID_ARG
