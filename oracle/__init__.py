@@ -64,7 +64,7 @@ def lib():
         _lib.oracle_pair_features.argtypes = [ctypes.POINTER(_Params), vp, vp, vp, vp, vp]
         _lib.oracle_attend.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, vp, vp]
         _lib.oracle_attend_blockwise.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, vp]
-        _lib.oracle_tri_attn.argtypes = [ctypes.POINTER(_Params), ci, vp, ci, vp, vp]
+        _lib.oracle_tri_attn.argtypes = [ctypes.POINTER(_Params), ci, vp, ci, vp, vp, vp]
         _lib.oracle_num_threads.restype = ci
     return _lib
 
@@ -196,10 +196,12 @@ def attend_blockwise(q, k, v, bias, mask=None, block=7):
     return o
 
 
-def tri_attn(p: Problem, orientation: int, lines=None, bias=None) -> np.ndarray:
+def tri_attn(p: Problem, orientation: int, lines=None, bias=None, want_o: bool = False):
     """The whole block.  orientation 0 (starting node): returns out[lines, :, :];
     orientation 1 (ending node): returns out[:, lines, :] laid out as
-    (len(lines), N, c_z), i.e. result[r, i] = out[i, lines[r]]."""
+    (len(lines), N, c_z), i.e. result[r, i] = out[i, lines[r]].
+    With want_o, returns (out, o): o is the attention output before the gate,
+    (len(lines), N, H, d), in the same line layout."""
     N, cz = p.N, p.c_z
     if lines is None:
         ln_arr, n = None, N
@@ -207,11 +209,13 @@ def tri_attn(p: Problem, orientation: int, lines=None, bias=None) -> np.ndarray:
         ln_arr = np.ascontiguousarray(np.asarray(lines, dtype=np.int32))
         n = len(ln_arr)
     out = np.empty((n, N, cz))
+    o = np.empty((n, N, p.H, p.d)) if want_o else None
     b = None if bias is None else _f64(bias)
     prm = p.params()
-    rc = lib().oracle_tri_attn(ctypes.byref(prm), int(orientation), _ptr(ln_arr), n, _ptr(b), _ptr(out))
+    rc = lib().oracle_tri_attn(ctypes.byref(prm), int(orientation), _ptr(ln_arr), n, _ptr(b),
+                               _ptr(out), _ptr(o))
     assert rc == 0, rc
-    return out
+    return (out, o) if want_o else out
 
 
 def tri_attn_full(p: Problem, orientation: int, bias=None) -> np.ndarray:

@@ -318,9 +318,11 @@ static int softmax_weighted_sum(double *s, const unsigned char *mask, long n,
   return 1;
 }
 
-/* Starting node, row i: out_row[j][c] = out_{i j c} for all j. */
+/* Starting node, row i: out_row[j][c] = out_{i j c} for all j; if o_row is
+ * not NULL, also o_row[j][h*d + c] = o_{i j h c}, the attention output before
+ * the gate. */
 static void start_row(const oracle_params *p, const double *bias_all, long i,
-                      double *out_row) {
+                      double *out_row, double *o_row) {
   long N = p->N;
   int H = p->H, d = p->d, HD = H * d, cz = p->c_z;
   double scale = 1.0 / sqrt((double)d);
@@ -349,6 +351,8 @@ static void start_row(const oracle_params *p, const double *bias_all, long i,
       /* o_ij = sum_k p_k v_ik */
       softmax_weighted_sum(s, p->mask, N, v + h * d, HD, d, o + h * d);
     }
+    if (o_row)
+      for (int t = 0; t < HD; ++t) o_row[j * HD + t] = o[t];
     for (int t = 0; t < HD; ++t) o[t] *= g[j * HD + t];
     linear(p->Wo, p->bo, o, cz, HD, upd);
     for (int c = 0; c < cz; ++c) out_row[j * cz + c] = z_at(p, i, j, c) + upd[c];
@@ -356,9 +360,11 @@ static void start_row(const oracle_params *p, const double *bias_all, long i,
   free(q); free(k); free(v); free(g); free(zb); free(xb); free(s); free(o); free(upd);
 }
 
-/* Ending node, column j: out_col[i][c] = out_{i j c} for all i. */
+/* Ending node, column j: out_col[i][c] = out_{i j c} for all i; if o_col is
+ * not NULL, also o_col[i][h*d + c] = o_{i j h c}, the attention output before
+ * the gate. */
 static void end_col(const oracle_params *p, const double *bias_all, long j,
-                    double *out_col) {
+                    double *out_col, double *o_col) {
   long N = p->N;
   int H = p->H, d = p->d, HD = H * d, cz = p->c_z;
   double scale = 1.0 / sqrt((double)d);
@@ -387,6 +393,8 @@ static void end_col(const oracle_params *p, const double *bias_all, long j,
       /* o_ij = sum_k p_k v_kj */
       softmax_weighted_sum(s, p->mask, N, v + h * d, HD, d, o + h * d);
     }
+    if (o_col)
+      for (int t = 0; t < HD; ++t) o_col[i * HD + t] = o[t];
     for (int t = 0; t < HD; ++t) o[t] *= g[i * HD + t];
     linear(p->Wo, p->bo, o, cz, HD, upd);
     for (int c = 0; c < cz; ++c) out_col[i * cz + c] = z_at(p, i, j, c) + upd[c];
@@ -399,9 +407,11 @@ static void end_col(const oracle_params *p, const double *bias_all, long j,
  *   orientation 1 (ending node):   lines are columns j; out[r][i][c] = out_{i, lines[r], c}
  * lines == NULL means every line 0..N-1 (n_lines must then be N).
  * bias_all may be NULL (computed here) or the [H][N][N] array produced by
- * oracle_pair_features, so repeated calls can share it. */
+ * oracle_pair_features, so repeated calls can share it.
+ * o_out may be NULL, or [n_lines][N][H*d]: the attention output o (before the
+ * gate) of the same pairs, laid out like out. */
 int oracle_tri_attn(const oracle_params *p, int orientation, const int *lines,
-                    int n_lines, const double *bias_all, double *out) {
+                    int n_lines, const double *bias_all, double *out, double *o_out) {
   if (!p || !out || p->N <= 0 || p->c_z <= 0 || p->H <= 0 || p->d <= 0)
     return -1;
   if (orientation != 0 && orientation != 1) return -1;
@@ -422,10 +432,11 @@ int oracle_tri_attn(const oracle_params *p, int orientation, const int *lines,
   for (int r = 0; r < n_lines; ++r) {
     long ln = lines ? lines[r] : r;
     double *dst = out + (long)r * N * p->c_z;
+    double *odst = o_out ? o_out + (long)r * N * p->H * p->d : NULL;
     if (orientation == 0)
-      start_row(p, bias_all, ln, dst);
+      start_row(p, bias_all, ln, dst, odst);
     else
-      end_col(p, bias_all, ln, dst);
+      end_col(p, bias_all, ln, dst, odst);
   }
   free(own);
   return 0;

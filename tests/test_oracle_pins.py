@@ -125,9 +125,12 @@ def test_probabilities_sum_to_one_masked_exactly_zero():
     assert np.all(P[:, :, m == 1] > 0.0)
 
 
-def _block_by_library(p: oracle.Problem, orientation: int) -> np.ndarray:
+def _block_by_library(p: oracle.Problem, orientation: int, want_o: bool = False):
     """The whole block composed from library routines (layer_norm, matmul,
-    sigmoid, scaled_dot_product_attention), for both orientations."""
+    sigmoid, scaled_dot_product_attention), for both orientations.  With
+    want_o, also the attention output before the gate, (line, N, H, d) in the
+    oracle's line layout (row a of the starting node, column a of the ending
+    node)."""
     T = torch.from_numpy
     N, H, d, cz = p.N, p.H, p.d, p.c_z
     z = T(np.asarray(p.Z, dtype=np.float64))
@@ -144,6 +147,7 @@ def _block_by_library(p: oracle.Problem, orientation: int) -> np.ndarray:
     if p.mask is not None:
         add[:, :, T(p.mask == 0)] = -math.inf
     out = torch.empty_like(z)
+    o_all = torch.empty(N, N, H, d, dtype=z.dtype)
     for a in range(N):
         # row a of the view: queries (a, j), keys (a, k), bias[h, j, k]
         o = F.scaled_dot_product_attention(q[a].permute(1, 0, 2), k[a].permute(1, 0, 2),
@@ -151,10 +155,11 @@ def _block_by_library(p: oracle.Problem, orientation: int) -> np.ndarray:
         o = o.permute(1, 0, 2).reshape(N, H * d)
         if p.mask is not None and not p.mask.any():
             o = torch.zeros_like(o)
+        o_all[a] = o.reshape(N, H, d)
         out[a] = z[a] + (g[a] * o) @ T(p.Wo).T + (T(p.bo) if p.bo is not None else 0.0)
     if orientation == 1:
         out = out.transpose(0, 1)
-    return out.numpy()
+    return (out.numpy(), o_all.numpy()) if want_o else out.numpy()
 
 
 @pytest.mark.parametrize("orientation", [0, 1])
@@ -165,6 +170,28 @@ def test_block_matches_library_composition(orientation, mask):
     got = oracle.tri_attn_full(p, orientation)
     ref = _block_by_library(p, orientation)
     np.testing.assert_allclose(got, ref, atol=1e-11)
+
+
+@pytest.mark.parametrize("orientation", [0, 1])
+@pytest.mark.parametrize("mask", ["none", "random:0.3"])
+def test_attention_output_matches_library_composition(orientation, mask):
+    """The attention output o (before the gate) that the oracle can return
+    beside out, against scaled_dot_product_attention in the composition, at
+    small widths and at the GPU widths, for every line and for a subset."""
+    inp, p = _small(N=10, seed=17, mask=mask)
+    p = _nonzero_biases(p)
+    _, o_ref = _block_by_library(p, orientation, want_o=True)
+    out, o = oracle.tri_attn(p, orientation, want_o=True)
+    np.testing.assert_allclose(o, o_ref, atol=1e-12)
+    lines = [7, 2, 9]
+    _, o_sub = oracle.tri_attn(p, orientation, lines, want_o=True)
+    np.testing.assert_allclose(o_sub, o_ref[lines], atol=1e-12)
+    inp = workloads.make_inputs(12, "bf16", 5, mask)
+    p64 = to_problem(inp)
+    p64.Z = inp.Z.to(torch.float64).numpy()
+    _, o_ref = _block_by_library(p64, orientation, want_o=True)
+    _, o = oracle.tri_attn(to_problem(inp), orientation, want_o=True)
+    np.testing.assert_allclose(o, o_ref, atol=1e-12)
 
 
 @pytest.mark.parametrize("orientation", [0, 1])
@@ -260,6 +287,12 @@ def test_zero_query_zero_bias_gives_masked_mean(orientation):
                 mean = v[valid, j].mean(0)   # keys (k, j)
             exp[i, j] = z[i, j] + p.Wo @ (g[i, j] * mean) + p.bo
     np.testing.assert_allclose(out, exp, atol=1e-12)
+    # the attention output itself, in the oracle's line layout
+    _, o = oracle.tri_attn(p, orientation, want_o=True)
+    for line in range(p.N):
+        mean = v[line, valid].mean(0) if orientation == 0 else v[valid, line].mean(0)
+        np.testing.assert_allclose(o[line].reshape(p.N, -1), np.broadcast_to(mean, (p.N, mean.size)),
+                                   atol=1e-12)
 
 
 def test_single_pair():
