@@ -50,8 +50,8 @@ NUM_SMS = 148
 SM_MAX_MHZ = 1965.0
 
 # DRAM bytes per tri_attn_fwd launch (starting node, N = 1536) from one ncu
-# capture (profiles/tri_attn_fwd_N1536.md), valid only for the kernel source
-# with this hash; otherwise reported as null.
+# capture of this kernel source, valid only for the source with this hash;
+# otherwise reported as null.
 TRAFFIC = {"tri_attn_fwd.cuh": "f9c788dbdbff8c0d", "bytes_per_launch": 1.832449e9 + 0.584904e9}
 
 

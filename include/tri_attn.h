@@ -62,9 +62,21 @@ extern "C" {
 /* ---- flags for tri_attn_forward --------------------------------------- */
 #define TRI_ATTN_FLAG_SYNC          1u  /* synchronise the stream and return the device status */
 #define TRI_ATTN_FLAG_TIME_KERNELS  2u  /* record CUDA events around each kernel (see tri_attn_kernel_times) */
-#define TRI_ATTN_FLAG_DEBUG_STALL   4u  /* fault injection: the attention kernel's producer withholds one
-                                           stage, so its consumers' bounded waits expire and the call
-                                           reports TRI_ATTN_ERR_TIMEOUT; nothing faults or traps */
+/* Fault injection, for tests of the error paths.  None of them faults, traps or
+ * hangs the GPU: a withheld copy makes the waiting threads' bounded waits
+ * (2 s) expire, those threads free what they hold and leave, and the call
+ * reports TRI_ATTN_ERR_TIMEOUT through the device status; the handle and the
+ * CUDA context stay usable. */
+#define TRI_ATTN_FLAG_DEBUG_STALL   4u  /* tri_attn_fwd: one CTA's producer withholds its first stage */
+#define TRI_ATTN_FLAG_DEBUG_STALL_PROJ 8u   /* pair_ln_proj: one group of one CTA never gets its first
+                                               tile of Z (every launch of the call) */
+#define TRI_ATTN_FLAG_DEBUG_STALL_GATE 16u  /* gate_out: one CTA's producer withholds its first stage
+                                               (every launch of the call) */
+#define TRI_ATTN_FLAG_DEBUG_FAIL_ALLOC 32u  /* if the call has to grow the handle's workspace, that
+                                               allocation fails as if cudaMalloc had run out of memory:
+                                               the call returns TRI_ATTN_ERR_OOM before any launch and
+                                               the handle holds no workspace afterwards (the old one is
+                                               released first); the next call allocates again */
 
 typedef enum { TRI_ATTN_F32 = 0, TRI_ATTN_BF16 = 1 } tri_attn_dtype;
 typedef enum { TRI_ATTN_STARTING = 0, TRI_ATTN_ENDING = 1 } tri_attn_orientation;
@@ -146,8 +158,8 @@ size_t tri_attn_workspace_bytes(tri_attn_dtype dtype, int N);
  * inspection by tests).  Layouts, for rows r of the last chunk and head h:
  *   q, k, v, g, o: [rows][H][N][d];  bias: [H][N][ld_bias]
  * (bias already scaled by log2(e); at masked keys and at columns >= N it is
- * -inf for F32 handles and -3e38 for BF16 handles, whose attention kernel adds
- * the bias with an MMA, where -inf would turn 0 * b into NaN;
+ * -inf for F32 handles and the finite -3e38 for BF16 handles, which keeps the
+ * sums it enters finite and still gives those keys probability exactly 0;
  * q already scaled by log2(e)/sqrt(d)).  Element type: bf16 for a BF16
  * handle, fp32 for F32.  Any output pointer may be NULL. */
 int tri_attn_debug_workspace(tri_attn_handle *h, void **q, void **k, void **v, void **g,
@@ -216,7 +228,7 @@ int tri_attn_rows_forward(tri_attn_handle *h, const void *Z_rows, int N, int row
  * (the status word is cleared at the start of each call): calls that overlap on
  * the GPU, e.g. on two streams of the same device, race and corrupt each other;
  * serialise them.  Flags: TRI_ATTN_FLAG_SYNC synchronises the stream and returns
- * the device status; the other flags are ignored. */
+ * the device status; the timing and fault-injection flags are ignored. */
 int tri_attn_forward_noalloc(const tri_attn_params *params, const void *Z, int N,
                              const uint8_t *mask, tri_attn_orientation orientation, void *out,
                              void *stream, unsigned flags);

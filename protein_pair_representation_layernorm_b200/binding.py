@@ -28,6 +28,9 @@ TRI_ATTN_ERR_NO_DEVICE = -7
 TRI_ATTN_FLAG_SYNC = 1
 TRI_ATTN_FLAG_TIME_KERNELS = 2
 TRI_ATTN_FLAG_DEBUG_STALL = 4
+TRI_ATTN_FLAG_DEBUG_STALL_PROJ = 8
+TRI_ATTN_FLAG_DEBUG_STALL_GATE = 16
+TRI_ATTN_FLAG_DEBUG_FAIL_ALLOC = 32
 
 TRI_ATTN_F32 = 0
 TRI_ATTN_BF16 = 1

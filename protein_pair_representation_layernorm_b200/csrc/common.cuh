@@ -13,10 +13,10 @@ constexpr int kHeads = 4;       // attention heads
 constexpr int kD = 32;          // head width
 constexpr int kHD = kHeads * kD;
 constexpr float kLog2e = 1.4426950408889634f;
-// Logit bias of a masked (or padding) key in the bf16 path.  Finite on purpose:
-// the attention kernel adds the bias with an identity-matrix MMA, where the
-// zeros of the identity meet every bias entry of the tile, and 0 * (-inf) would
-// be NaN.  2^(kMaskedLogit - m) is exactly 0 in fp32 for any finite offset m.
+// Logit bias of a masked (or padding) key in the bf16 path.  Finite, so that
+// every sum it enters (score + bias, minus the running offset) stays a finite
+// number rather than an infinity; 2^(kMaskedLogit + s - m) is exactly 0 in
+// fp32 for any finite score s and offset m, so the key gets probability 0.
 constexpr float kMaskedLogit = -3.0e38f;
 
 // Offset (in elements) of pair (i, j) of the problem inside Z / out.  The
@@ -66,6 +66,7 @@ struct ProjArgs {
   // Z holds problem rows z_row0.. (a row slab; 0 for the whole tensor), and the
   // bias buffer holds, per head, bias_rows problem rows starting at bias_row0
   int z_row0, bias_row0, bias_rows;
+  int debug_stall;  // fault injection: group 0 of CTA 0 never gets its first tile of Z
   int* status;
 };
 
@@ -83,6 +84,7 @@ struct GateArgs {
   __nv_bfloat16* out;
   int N, orient, row0, rows;
   int z_row0;  // Z and out hold problem rows z_row0.. (a row slab; 0 for the whole tensor)
+  int debug_stall;  // fault injection: the producer of CTA 0 withholds its first stage
   int* status;
 };
 

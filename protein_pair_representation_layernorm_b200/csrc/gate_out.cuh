@@ -107,6 +107,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&map_z);
       mbar_arrive_expect_tx(w_bar, kWoBytes);
       bulk_load(smem + kSmemW, a.wo_img, kWoBytes, w_bar);
+      // fault injection: CTA 0 never fills its first stage, so the compute
+      // threads' bounded wait expires and the launch reports TRI_ATTN_ERR_TIMEOUT
+      const bool stall = a.debug_stall && blockIdx.x == 0;
       long long n_issued = 0;
       for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++n_issued) {
         const int s = static_cast<int>(n_issued % kStages);
@@ -117,6 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           report_status(a.status, kStatusTimeout);
           break;
         }
+        if (stall && n_issued == 0) continue;
         uint8_t* st = smem + kSmemStages + s * kStageBytes;
         const int r = static_cast<int>(tile / jtiles);
         const int j0 = static_cast<int>(tile % jtiles) * kTileM;
@@ -133,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // never leave a copy in flight into this CTA's shared memory
       if (!mbar_wait(w_bar, 0, nullptr)) report_status(a.status, kStatusTimeout);
       for (long long n = n_issued - kStages; n < n_issued; ++n)
-        if (n >= 0 &&
+        if (n >= 0 && !(stall && n == 0) &&
             !mbar_wait(&full[n % kStages], static_cast<uint32_t>(n / kStages) & 1, nullptr))
           report_status(a.status, kStatusTimeout);
     }

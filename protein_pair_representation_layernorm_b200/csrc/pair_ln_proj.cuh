@@ -127,9 +127,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_load_3d(sA + kAAtomBytes, &map_z, &z_full[grp], 64, c1, c2);
   };
   if (mma_thread) tma_prefetch_desc(&map_z);
-  if (mma_thread && tile < ntiles) issue_z(tile);
+  // fault injection: group 0 of CTA 0 never receives its first tile, so its
+  // bounded wait below expires and the launch reports TRI_ATTN_ERR_TIMEOUT
+  const bool stall = a.debug_stall && blockIdx.x == 0 && grp == 0;
+  if (mma_thread && tile < ntiles && !stall) issue_z(tile);
   uint32_t z_phase = 0;
-  bool z_pending = tile < ntiles;
+  bool z_pending = tile < ntiles && !stall;
   for (; tile < ntiles; tile += stride) {
     const int r = static_cast<int>(tile / jtiles);
     const int i = a.row0 + r;

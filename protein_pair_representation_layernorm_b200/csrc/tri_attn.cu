@@ -265,11 +265,18 @@ Layout layout_for(tri_attn_dtype dt, int N, int rows) {
   return L;
 }
 
-int ensure_workspace(tri_attn_handle* h, size_t bytes) {
+// Grow the workspace to `bytes`.  The old buffer is released first, so a
+// failed allocation leaves the handle holding no workspace (and nothing
+// leaked); the next call allocates again.  fail_alloc injects that failure.
+int ensure_workspace(tri_attn_handle* h, size_t bytes, bool fail_alloc = false) {
   if (h->ws_bytes >= bytes) return TRI_ATTN_OK;
-  if (h->ws) cudaFree(h->ws);
+  if (h->ws) CUDA_TRY(cudaFree(h->ws));
   h->ws = nullptr;
   h->ws_bytes = 0;
+  if (fail_alloc) {
+    TA_LOG("workspace allocation of %zu bytes failed (injected)", bytes);
+    return TRI_ATTN_ERR_OOM;
+  }
   CUDA_TRY(cudaMalloc(&h->ws, bytes));
   h->ws_bytes = bytes;
   return TRI_ATTN_OK;
@@ -355,8 +362,12 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
   if (hook && hook->max_rows > 0 && hook->max_rows < rows) rows = hook->max_rows;
   const bool chunked = rows < zrows;
   const Layout L = layout_for(dt, N, rows);
-  int rc = ensure_workspace(h, L.total);
-  if (rc != TRI_ATTN_OK) return rc;
+  int rc = ensure_workspace(h, L.total, (flags & TRI_ATTN_FLAG_DEBUG_FAIL_ALLOC) != 0);
+  if (rc != TRI_ATTN_OK) {
+    h->q = h->k = h->v = h->g = h->o = h->bias = nullptr;  // the old workspace is gone
+    h->rows_last = 0;
+    return rc;
+  }
   char* ws = static_cast<char*>(h->ws);
   h->q = ws + L.q;
   h->k = ws + L.k;
@@ -486,6 +497,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
     a.z_row0 = rbeg;
     a.bias_row0 = slab && slab->phase == 0 ? rbeg : 0;
     a.bias_rows = slab && slab->phase == 0 ? zrows : N;
+    a.debug_stall = (flags & TRI_ATTN_FLAG_DEBUG_STALL_PROJ) ? 1 : 0;
     a.status = h->status;
     const long long ntiles = static_cast<long long>(nrows) * jtiles;
     const unsigned grid = static_cast<unsigned>(
@@ -584,6 +596,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
       a.row0 = r0;
       a.rows = nr;
       a.z_row0 = rbeg;
+      a.debug_stall = (flags & TRI_ATTN_FLAG_DEBUG_STALL_GATE) ? 1 : 0;
       a.status = h->status;
       const long long ntiles = static_cast<long long>(nr) * jtiles;
       const unsigned grid = static_cast<unsigned>(std::min<long long>(ntiles, h->num_sms));
@@ -665,8 +678,12 @@ int tri_attn_create(const tri_attn_params* p, tri_attn_handle** out) {
     tri_attn_destroy(h);
     return code;
   };
-  cudaGetDevice(&h->device);
-  cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+  if (cudaGetDevice(&h->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return fail(TRI_ATTN_ERR_CUDA);
+  }
   h->dtype = p->dtype;
   h->eps = p->ln_eps;
   h->q_scale = tri::kLog2e / std::sqrt(static_cast<float>(kD));
@@ -1121,7 +1138,7 @@ extern "C" int tri_attn_forward_noalloc(const tri_attn_params* p, const void* Z,
   // forward below never reaches cudaMalloc
   tri_attn_handle hh;
   hh.device = dev;
-  cudaDeviceGetAttribute(&hh.num_sms, cudaDevAttrMultiProcessorCount, dev);
+  CUDA_TRY(cudaDeviceGetAttribute(&hh.num_sms, cudaDevAttrMultiProcessorCount, dev));
   hh.dtype = TRI_ATTN_BF16;
   hh.eps = p->ln_eps;
   hh.q_scale = tri::kLog2e / std::sqrt(static_cast<float>(kD));
@@ -1137,7 +1154,7 @@ extern "C" int tri_attn_forward_noalloc(const tri_attn_params* p, const void* Z,
   hh.ws_bytes = kNoallocScratchBytes - kNaWs;
   hh.ws_limit = hh.ws_bytes;
   rc = forward_impl(&hh, Z, N, mask, static_cast<int>(orientation), out, st,
-                    flags & ~(TRI_ATTN_FLAG_TIME_KERNELS | TRI_ATTN_FLAG_DEBUG_STALL));
+                    flags & TRI_ATTN_FLAG_SYNC);
   if (rc == TRI_ATTN_OK && (flags & TRI_ATTN_FLAG_SYNC)) {
     int s = 0;
     CUDA_TRY(cudaMemcpyAsync(&s, hh.status, sizeof(int), cudaMemcpyDeviceToHost, st));

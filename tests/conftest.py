@@ -10,6 +10,18 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """One line per GPU parity comparison (errors and lines compared)."""
+    try:
+        from gpu_util import PARITY_LOG
+    except Exception:
+        return
+    if PARITY_LOG:
+        terminalreporter.section("parity against the oracle")
+        for line in PARITY_LOG:
+            terminalreporter.write_line(line)
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU oracle case")

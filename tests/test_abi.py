@@ -103,3 +103,13 @@ def test_row_slab_calls_reject_bad_arguments_without_device():
         binding.TRI_ATTN_ERR_INVALID_ARG
     assert L.tri_attn_rows_forward(None, buf, 16, 0, 16, None, buf, buf, None, 0) == \
         binding.TRI_ATTN_ERR_INVALID_ARG
+
+
+def test_binding_constants_match_the_header():
+    """Every status code and flag the header defines has the same value in the binding."""
+    with open(os.path.join(ROOT, "include", "tri_attn.h")) as f:
+        text = f.read()
+    defs = re.findall(r"#define\s+(TRI_ATTN_(?:OK|ERR_\w+|FLAG_\w+))\s+(-?\d+)u?", text)
+    assert len(defs) >= 14
+    for name, value in defs:
+        assert getattr(binding, name) == int(value), name

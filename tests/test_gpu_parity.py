@@ -2,51 +2,93 @@
 inputs, through the C ABI.
 
 Tolerances (on out): fp32 inputs max-abs 1e-4; bf16 inputs with fp32
-accumulation rel-L2 5e-3 and max-abs 2e-2.  Full tensors where the oracle
-finishes in seconds; at the large workloads the oracle evaluates sampled
-lines (rows for the starting node, columns for the ending node) one by one,
-in the same launch configuration the benchmark times.
+accumulation rel-L2 5e-3 and max-abs 2e-2.  The attention update is held to
+rel-L2 2e-2 as well: the GPU's attention output o (before the gate, read from
+the workspace) against the oracle's, at every bf16 workload and both
+orientations; and out - z against oracle - z on inputs scaled by 2^-4 (exact
+in bf16; LayerNorm leaves the update almost unchanged while the residual
+shrinks sixteenfold, so the bf16 rounding of out no longer hides the update).
+Full tensors where the oracle finishes in seconds; at the large workloads the
+oracle evaluates sampled lines (rows for the starting node, columns for the
+ending node) one by one, in the same launch configuration the benchmark
+times.
 """
+import functools
+
 import numpy as np
 import pytest
 import torch
 
 import oracle
 from conftest import to_problem
-from gpu_util import (assert_within, block_for, compare, lines_of, run_gpu, z_lines)
+from gpu_util import (assert_within, attn_output_lines, block_for, compare, lines_of,
+                      log_parity, run_gpu, z_lines)
 from protein_pair_representation_layernorm_b200 import binding, workloads
 
 pytestmark = pytest.mark.gpu
 
+NAMES = {0: "starting", 1: "ending"}
 
-def _check_full(inp, orientation, dtype, what):
-    out, _ = run_gpu(inp, orientation)
+
+def _check_full(inp, orientation, dtype, what, with_o=True):
+    out, blk = run_gpu(inp, orientation)
     p = to_problem(inp)
-    ref = oracle.tri_attn_full(p, orientation)
-    st = compare(out.double().cpu().numpy(), ref, inp.Z.double().numpy(), dtype)
+    if dtype == "bf16" and with_o:
+        ref, ref_o = oracle.tri_attn(p, orientation, want_o=True)
+        got_o = attn_output_lines(blk, inp.N, range(inp.N))
+    else:
+        ref, ref_o, got_o = oracle.tri_attn(p, orientation), None, None
+    if orientation == 1:
+        ref = np.ascontiguousarray(ref.transpose(1, 0, 2))
+    st = compare(out.double().cpu().numpy(), ref, inp.Z.double().numpy(), dtype, got_o, ref_o)
     assert_within(st, dtype, what)
+    log_parity(what, st, inp.N)
     return st
 
 
-def _check_lines(inp, orientation, lines, dtype, what, out=None):
-    if out is None:
-        out, _ = run_gpu(inp, orientation)
+def _check_lines(inp, orientation, lines, dtype, what, update_at_out=False):
+    out, blk = run_gpu(inp, orientation)
     p = to_problem(inp)
     bias = oracle.bias_all(p)
-    ref = oracle.tri_attn(p, orientation, lines, bias=bias)
+    ref, ref_o = oracle.tri_attn(p, orientation, lines, bias=bias, want_o=True)
     got = lines_of(out, orientation, lines)
-    st = compare(got, ref, z_lines(inp.Z, orientation, lines), dtype)
-    assert_within(st, dtype, what)
+    got_o = attn_output_lines(blk, inp.N, lines)
+    st = compare(got, ref, z_lines(inp.Z, orientation, lines), dtype, got_o, ref_o)
+    assert_within(st, dtype, what, update_at_out=update_at_out)
+    log_parity(what, st, len(lines))
+    blk.close()
     return st
 
 
-def _sample_lines(N, n, seed):
+def _sample_lines(N, n, seed, extra=()):
+    """n distinct lines: 0, N-1, N/2, the extra ones, the rest seeded random."""
     rng = np.random.default_rng(seed)
-    fixed = [0, N - 1, N // 2]
-    rest = rng.choice(N, size=min(N, n) - len(fixed), replace=False).tolist()
-    return sorted(set(fixed + rest))
+    fixed = sorted(set([0, N - 1, N // 2] + [int(x) for x in extra]))
+    pool = np.setdiff1d(np.arange(N), fixed)
+    rest = rng.choice(pool, size=max(0, min(N, n) - len(fixed)), replace=False).tolist()
+    return sorted(fixed + rest)
 
 
+@functools.lru_cache(maxsize=1)
+def _workload(w: int, scale_pow2: int = 0):
+    inp = workloads.workload_inputs(w)
+    if scale_pow2:
+        # exact in bf16 (a power of two; no value of these workloads comes near underflow)
+        inp = workloads.Inputs(Z=inp.Z * (2.0 ** scale_pow2), **{k: getattr(inp, k) for k in (
+            "mask", "gamma", "beta", "Wq", "Wk", "Wv", "Wg", "bg", "Wb", "Wo", "bo")})
+    return inp
+
+
+def _lines_for(w: int, inp):
+    N = inp.N
+    if w == 2:  # rows spanning all three chains, chain boundaries included
+        return _sample_lines(N, 24, 2, extra=[255, 256, 511, 512])
+    if w == 3:
+        return _sample_lines(N, 32, 3, extra=[127, 128, 1535 - 63])
+    if w == 4:  # masked residues among the lines
+        masked = np.flatnonzero(inp.mask.numpy() == 0)
+        return _sample_lines(N, 32, 4, extra=masked[:3].tolist() + [4095 - 64])
+    raise ValueError(w)
 def test_workload0_fp32_full():
     inp = workloads.workload_inputs(0)
     _check_full(inp, 0, "f32", "workload 0")
@@ -55,30 +97,27 @@ def test_workload0_fp32_full():
 @pytest.mark.parametrize("orientation", [0, 1])
 def test_workload1_full(orientation):
     inp = workloads.workload_inputs(1)
-    _check_full(inp, orientation, "bf16", f"workload 1 orient {orientation}")
+    _check_full(inp, orientation, "bf16", f"workload 1 (N=384) {NAMES[orientation]}")
 
 
 @pytest.mark.parametrize("orientation", [0, 1])
-def test_workload2_sampled(orientation):
-    inp = workloads.workload_inputs(2)
-    # rows spanning all three chains, chain boundaries included
-    lines = sorted(set(_sample_lines(768, 16, 2) + [255, 256, 511, 512]))
-    _check_lines(inp, orientation, lines, "bf16", f"workload 2 orient {orientation}")
+@pytest.mark.parametrize("w", [2, 3, 4])
+def test_workload_sampled(w, orientation):
+    inp = _workload(w)
+    lines = _lines_for(w, inp)
+    _check_lines(inp, orientation, lines, "bf16", f"workload {w} (N={inp.N}) {NAMES[orientation]}")
 
 
 @pytest.mark.parametrize("orientation", [0, 1])
-def test_workload3_sampled(orientation):
-    inp = workloads.workload_inputs(3)
-    _check_lines(inp, orientation, _sample_lines(1536, 8, 3), "bf16",
-                 f"workload 3 orient {orientation}")
-
-
-@pytest.mark.parametrize("orientation", [0, 1])
-def test_workload4_sampled(orientation):
-    inp = workloads.workload_inputs(4)
-    masked = np.flatnonzero(inp.mask.numpy() == 0)
-    lines = sorted(set(_sample_lines(4096, 5, 4) + [int(masked[0])]))
-    _check_lines(inp, orientation, lines, "bf16", f"workload 4 orient {orientation}")
+@pytest.mark.parametrize("w", [1, 2, 3, 4])
+def test_update_small_residual(w, orientation):
+    """The attention update asserted at out level: the workload's Z times 2^-4,
+    so out - z is no longer dwarfed by z and the update error is measured
+    through every kernel, gate and output projection included."""
+    inp = _workload(w, scale_pow2=-4)
+    lines = list(range(inp.N)) if w == 1 else _lines_for(w, inp)
+    _check_lines(inp, orientation, lines, "bf16",
+                 f"workload {w} (N={inp.N}) x 2^-4 {NAMES[orientation]}", update_at_out=True)
 
 
 # key-tile counts T = ceil(N / 64): 1, 1, 2, 3, 4, 5, 7 (the attention kernel's
