@@ -76,32 +76,50 @@ class ShardedTriangleAttention:
         return self.block.rows_forward(Z_rows, N, row0, bias_all, mask)
 
     def gather_bias(self, bias_rows: torch.Tensor, N: int) -> torch.Tensor:
-        """All-gather of every rank's bias rows into the whole [H][N][ld] bias
-        (one all-gather per head, each slab padded to S rows)."""
+        """All-gather of every rank's bias rows into the whole [H][N][ld] bias:
+        one all_gather_into_tensor over the slab-major layout [world][H][S][ld]
+        (each rank's slab padded to S rows only if it has fewer), then one
+        strided copy into the head-major layout the attention kernel reads."""
         H, nrows, ld = bias_rows.shape
         S = -(-N // self.world)
+        mine = bias_rows
+        if nrows < S or not bias_rows.is_contiguous():
+            mine = torch.zeros(H, S, ld, dtype=bias_rows.dtype, device=bias_rows.device)
+            mine[:, :nrows] = bias_rows
+        flat = torch.empty(self.world * H, S, ld, dtype=bias_rows.dtype, device=bias_rows.device)
+        dist.all_gather_into_tensor(flat, mine.contiguous(), group=self.group)
+        gathered = flat.view(self.world, H, S, ld)
         out = torch.empty(H, N, ld, dtype=bias_rows.dtype, device=bias_rows.device)
-        for h in range(H):
-            mine = torch.zeros(S, ld, dtype=bias_rows.dtype, device=bias_rows.device)
-            mine[:nrows] = bias_rows[h]
-            parts = [torch.empty_like(mine) for _ in range(self.world)]
-            dist.all_gather(parts, mine, group=self.group)
-            out[h] = torch.cat(parts, dim=0)[:N]
+        # rank p's rows are p*S .. p*S+S-1: out[h][p*S + r] = gathered[p][h][r]
+        full = out.view(H, N, ld) if self.world * S == N else None
+        if full is not None:
+            full.view(H, self.world, S, ld).copy_(gathered.permute(1, 0, 2, 3))
+        else:
+            out.copy_(gathered.permute(1, 0, 2, 3).reshape(H, self.world * S, ld)[:, :N])
         return out
 
     def transpose_rows(self, X_rows: torch.Tensor, N: int) -> torch.Tensor:
         """This rank's rows of the transpose (pair (i, j) -> (j, i)) of a row-
-        sharded N x N x C tensor, by one all-to-all of S x S blocks."""
+        sharded N x N x C tensor, by one all-to-all of S x S blocks.  Block q of
+        the send buffer is X[my rows][rows of q]; it is packed with one strided
+        copy (X viewed as [S][world][S][C], columns padded to world*S when N is
+        not a multiple of the world size) and unpacked with another."""
         shards = row_shards(N, self.world)
         S = -(-N // self.world)
         row0, nrows = shards[self.rank]
         C = X_rows.shape[2]
-        send = torch.zeros(self.world, S, S, C, dtype=X_rows.dtype, device=X_rows.device)
-        for q, (c0, nc) in enumerate(shards):
-            send[q, :nrows, :nc] = X_rows[:, c0:c0 + nc]           # X[R_me][R_q]
+        W = self.world
+        if nrows == S and W * S == N:
+            src = X_rows.view(S, W, S, C)
+        else:
+            src = torch.zeros(S, W * S, C, dtype=X_rows.dtype, device=X_rows.device)
+            src[:nrows, :N] = X_rows
+            src = src.view(S, W, S, C)
+        send = src.permute(1, 0, 2, 3).contiguous()                # [q][my row][col of q]
         recv = torch.empty_like(send)
         dist.all_to_all_single(recv, send, group=self.group)       # block p = X[R_p][R_me]
-        out = torch.empty(nrows, N, C, dtype=X_rows.dtype, device=X_rows.device)
-        for p, (c0, nc) in enumerate(shards):
-            out[:, c0:c0 + nc] = recv[p, :nc, :nrows].transpose(0, 1)
-        return out.contiguous()
+        # out[c][p*S + i] = recv[p][i][c]
+        t = recv.permute(2, 0, 1, 3)                               # [my col][p][row of p]
+        if nrows == S and W * S == N:
+            return t.reshape(S, N, C).contiguous()
+        return t.reshape(S, W * S, C)[:nrows, :N].contiguous()
