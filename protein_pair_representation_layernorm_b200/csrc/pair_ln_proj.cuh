@@ -1,27 +1,36 @@
 // pair_ln_proj.cuh — LayerNorm + fused Q/K/V/gate projection (tcgen05) + logit
 // bias, bf16 pair representation.
 //
-// Persistent CTAs of two independent 128-thread groups.  Each group walks its
+// Persistent CTAs of two independent groups of 8 warps.  Each group walks its
 // own tiles of 128 pairs of one problem row (pairs (i, j0..j0+127)).  The tile of
 // Z arrives by TMA straight into the group's MMA A buffer (K-major, 128-byte
 // swizzle: two boxes of 64 channels; the ending-node block reads the swapped
 // view, pair (i, j) = Z[j][i], as a box one pair wide and 128 pairs deep).
-// Thread t of the group owns pair j0+t:
-//   1. reads its 256-byte pair vector from the buffer,
-//   2. LayerNorm in fp32 (mean, biased variance, rsqrt),
-//   3. the per-head logit bias  Wb x  in fp32 (Wb pre-scaled by log2 e;
-//      kMaskedLogit at masked keys and at the padding columns j >= N),
-//   4. writes x as bf16 back in place, which makes the buffer the A operand.
-// The next tile's TMA is issued as soon as the projection has consumed the
-// buffer, so it overlaps the last epilogue.
+// Two threads share a pair: warp w of the group (w = 0..7) owns the pairs
+// 32 (w % 4) .. +31 (its TMEM lane quadrant) and the channel half w / 4, which
+// is exactly one 64-channel box of the A buffer.  Per tile each thread
+//   1. reads its 64 channels (128 B) from the buffer,
+//   2. sums, in one pass, z - K and (z - K)^2 (K = channel 0 of the pair, a
+//      shift that keeps the variance free of cancellation) and the four logit-
+//      bias dot products Wb gamma (z - K) (Wb pre-scaled by log2 e),
+//   3. exchanges these six partial sums with the other thread of its pair
+//      through shared memory (both add them in the same order, so the two
+//      agree bit for bit), which gives the mean, the biased variance, rsqrt,
+//      and the bias  rstd (S_h - (mean - K) sum_c Wb gamma) + Wb beta,
+//      kMaskedLogit at masked keys and at the padding columns j >= N,
+//   4. writes its normalised channels as bf16 back in place, which makes the
+//      buffer the A operand.
 // One thread of the group then issues the projection D = X W^T in two halves of
 // N = 256 (q|k, then v|g), W = [Wq; Wk; Wv; Wg] resident in shared memory for the
-// whole kernel, each half accumulating in fp32 in the group's 256 TMEM columns.
-// Each thread reads back its TMEM lane; q (scaled by log2(e)/sqrt(d)), k, v and
-// sigmoid(g + bg) are written head-major ([rows][H][N][d], bf16): each warp
-// stages its 32 pairs' 64-byte rows of one head in shared memory and writes
-// them with one TMA store (a contiguous 2 KB block).  While one group runs its MMAs the other normalises or
-// stores, so the tensor core, the ALUs and HBM overlap.
+// whole kernel, each half accumulating in fp32 in the group's 256 TMEM columns;
+// the next tile's TMA is issued as soon as the second half has consumed the
+// buffer.  In the epilogue of a half the two threads of a pair take one output
+// each (q or k, v or g): the thread reads its TMEM lane, scales q by
+// log2(e)/sqrt(d), forms sigmoid(g + bg), and writes the pair's 64-byte row of
+// each head of the head-major output ([rows][H][N][d], bf16) with two 32-byte
+// stores straight from registers (a warp's 32 pairs fill a contiguous 2 KB
+// block).  While one group runs its MMAs the other normalises or stores, so the
+// tensor core, the ALUs and HBM overlap.
 //
 // This is the HBM-bound step: per pair it reads 256 B and writes 1 KB + 8 B.
 #pragma once
@@ -32,7 +41,7 @@
 namespace tri {
 namespace plp {
 
-constexpr int kGroupThreads = 128;
+constexpr int kGroupThreads = 256;                   // two threads per pair
 constexpr int kGroupsPerCta = 2;
 constexpr int kThreads = kGroupThreads * kGroupsPerCta;
 constexpr int kTileM = 128;
@@ -40,47 +49,72 @@ constexpr int kNOut = 4 * kHD;                       // q | k | v | g
 constexpr uint32_t kWImgBytes = kNOut * kCz * 2;     // 131072
 constexpr uint32_t kWAtomBytes = kNOut * 128;        // one 64-element K slab of W
 constexpr uint32_t kATileBytes = kTileM * kCz * 2;   // 32768
-constexpr uint32_t kAAtomBytes = kTileM * 128;       // 16384
+constexpr uint32_t kAAtomBytes = kTileM * 128;       // 16384: one 64-channel box
 constexpr uint32_t kSmemW = 0;
 constexpr uint32_t kSmemA = kWImgBytes;                                  // + grp * kATileBytes
 constexpr uint32_t kSmemPar = kSmemA + kGroupsPerCta * kATileBytes;     // fp32 params
-constexpr uint32_t kParFloats = kHeads * kCz + 3 * kCz;                 // w_b, gamma, beta, b_g
-constexpr uint32_t kSmemStg = kSmemPar + kParFloats * 4;               // per-warp store staging
-constexpr uint32_t kStgBytes = 32 * 64;                                 // 32 pairs x 64 B
-constexpr uint32_t kSmemBar = kSmemStg + (kThreads / 32) * kStgBytes;
+// w_b * gamma [H][c_z], gamma, beta, b_g, then per head sum_c w_b gamma and w_b . beta
+constexpr uint32_t kParFloats = kHeads * kCz + 3 * kCz + 2 * kHeads;
+constexpr int kPartials = 2 + kHeads;                // sum, sum of squares, 4 bias dots
+constexpr uint32_t kSmemXch = kSmemPar + ((kParFloats * 4 + 15) / 16) * 16;
+// [group][channel half][partial][pair]
+constexpr uint32_t kXchBytes = kGroupsPerCta * 2 * kPartials * kTileM * 4;
+constexpr uint32_t kSmemBar = kSmemXch + kXchBytes;
 constexpr uint32_t kSmemBytes = kSmemBar + 64 + 1024;                   // + alignment slack
 static_assert(kGroupsPerCta * 2 * 8 + 8 + 8 <= 64, "barrier area");
 constexpr uint32_t kTmemCols = 512;                                     // 256 per group
 
 __global__ void __launch_bounds__(kThreads, 1)
-    pair_ln_proj(const __grid_constant__ CUtensorMap map_z, const __grid_constant__ CUtensorMap map_q,
-                 const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
-                 const __grid_constant__ CUtensorMap map_g, const ProjArgs a) {
+    pair_ln_proj(const __grid_constant__ CUtensorMap map_z, const ProjArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  float* s_wb = reinterpret_cast<float*>(smem + kSmemPar);
-  float* s_gamma = s_wb + kHeads * kCz;
+  float* s_wbg = reinterpret_cast<float*>(smem + kSmemPar);  // w_b[h][c] * gamma[c]
+  float* s_gamma = s_wbg + kHeads * kCz;
   float* s_beta = s_gamma + kCz;
   float* s_bg = s_beta + kCz;
+  float* s_wsum = s_bg + kCz;        // [h]: sum_c w_b[h][c] gamma[c]
+  float* s_wbeta = s_wsum + kHeads;  // [h]: sum_c w_b[h][c] beta[c]
+  float* s_xch = reinterpret_cast<float*>(smem + kSmemXch);
   uint64_t* w_bar = reinterpret_cast<uint64_t*>(smem + kSmemBar);
   uint64_t* mma_bar = w_bar + 1;                // one per group
   uint64_t* z_full = mma_bar + kGroupsPerCta;   // one per group
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(z_full + kGroupsPerCta);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int grp = tid / kGroupThreads;
-  const int gt = tid % kGroupThreads;           // pair within the tile = TMEM lane
+  const int gt = tid % kGroupThreads;
+  const int wq = (warp % 8) & 3;                // TMEM lane quadrant
+  const int hc = (warp % 8) >> 2;               // channel half (LN) / output of a half (epilogue)
+  const int p = wq * 32 + lane;                 // pair within the tile = TMEM lane
   const uint32_t bar_id = 1 + grp;
   const bool qkvg = a.write_qkvg != 0;
   uint8_t* sA = smem + kSmemA + grp * kATileBytes;
 
-  for (int idx = tid; idx < kHeads * kCz; idx += kThreads) s_wb[idx] = a.w_b[idx];
+  for (int idx = tid; idx < kHeads * kCz; idx += kThreads)
+    s_wbg[idx] = a.w_b[idx] * a.gamma[idx % kCz];
   for (int idx = tid; idx < kCz; idx += kThreads) {
     s_gamma[idx] = a.gamma[idx];
     s_beta[idx] = a.beta[idx];
     s_bg[idx] = a.b_g[idx];
+  }
+  if (warp < kHeads) {  // per-head constants of the bias: one warp per head
+    float sw = 0.f, sb = 0.f;
+    for (int c = lane; c < kCz; c += 32) {
+      const float w = a.w_b[warp * kCz + c];
+      sw = fmaf(w, a.gamma[c], sw);
+      sb = fmaf(w, a.beta[c], sb);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sw += __shfl_xor_sync(0xffffffffu, sw, o);
+      sb += __shfl_xor_sync(0xffffffffu, sb, o);
+    }
+    if (lane == 0) {
+      s_wsum[warp] = sw;
+      s_wbeta[warp] = sb;
+    }
   }
   if (tid == 0) {
     mbar_init(w_bar, 1);
@@ -109,11 +143,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long ntiles = static_cast<long long>(a.rows) * jtiles;
   const long long stride = static_cast<long long>(gridDim.x) * kGroupsPerCta;
   const uint32_t sA_u32 = smem_u32(sA), sW_u32 = smem_u32(smem + kSmemW);
-  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
   constexpr uint32_t kIdesc = idesc_bf16_f32(128, 256, false);
   uint32_t mma_phase = 0;
   bool w_ready = false;
   const bool mma_thread = gt == 0;
+  // the group's exchange area: [channel half][partial][pair]
+  float* xch = s_xch + grp * (2 * kPartials * kTileM);
+  uint8_t* row = sA + hc * kAAtomBytes + p * 128;  // this thread's 64 channels
 
   long long tile = static_cast<long long>(blockIdx.x) * kGroupsPerCta + grp;
   // TMA of a tile of Z into this group's A buffer
@@ -136,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (; tile < ntiles; tile += stride) {
     const int r = static_cast<int>(tile / jtiles);
     const int i = a.row0 + r;
-    const int j = static_cast<int>(tile % jtiles) * kTileM + gt;
+    const int j = static_cast<int>(tile % jtiles) * kTileM + p;
     const bool jv = j < a.N;
 
     if (!named_barrier_and(bar_id, kGroupThreads, mbar_wait(&z_full[grp], z_phase, abort_flag))) {
@@ -145,95 +182,111 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     z_phase ^= 1;
     z_pending = false;
-    uint4 zr[16];
+    // this thread's 64 channels: 16-byte chunk c of the row sits at c ^ (p % 8)
+    uint4 zr[8];
 #pragma unroll
-    for (int c = 0; c < 16; ++c)
-      zr[c] = *reinterpret_cast<const uint4*>(sA + (c >> 3) * kAAtomBytes + gt * 128 +
-                                              (((c & 7) ^ (gt & 7)) << 4));
+    for (int c = 0; c < 8; ++c)
+      zr[c] = *reinterpret_cast<const uint4*>(row + ((c ^ (p & 7)) << 4));
+    // the shift K: channel 0 of the pair (first bf16 of chunk 0 of the first box)
+    const float K =
+        bf16lo_to_f32(*reinterpret_cast<const uint32_t*>(sA + p * 128 + ((p & 7) << 4)));
 
-    // ---- LayerNorm statistics in fp32: two passes over registers, packed
-    // fp32x2 arithmetic on channel pairs, two independent accumulators each
+    // ---- one pass: sum of (z - K), of (z - K)^2 and the four bias dot products
     auto chan2 = [](uint32_t w) { return make_float2(bf16lo_to_f32(w), bf16hi_to_f32(w)); };
-    float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    const float2 nK = make_float2(-K, -K);
+    float2 s1[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    float2 sb[kHeads] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
+    const float4* w4 = reinterpret_cast<const float4*>(s_wbg);
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      acc[0] = __fadd2_rn(acc[0], chan2(zr[c].x));
-      acc[1] = __fadd2_rn(acc[1], chan2(zr[c].y));
-      acc[0] = __fadd2_rn(acc[0], chan2(zr[c].z));
-      acc[1] = __fadd2_rn(acc[1], chan2(zr[c].w));
-    }
-    const float mu = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) * (1.0f / kCz);
-    const float2 nmu = make_float2(-mu, -mu);
-    acc[0] = acc[1] = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
+    for (int c = 0; c < 8; ++c) {
       const uint32_t w[4] = {zr[c].x, zr[c].y, zr[c].z, zr[c].w};
+      float2 d[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float2 d = __fadd2_rn(chan2(w[e]), nmu);
-        acc[e & 1] = __ffma2_rn(d, d, acc[e & 1]);
+        d[e] = __fadd2_rn(chan2(w[e]), nK);
+        s1[e & 1] = __fadd2_rn(s1[e & 1], d[e]);
+        s2[e & 1] = __ffma2_rn(d[e], d[e], s2[e & 1]);
       }
-    }
-    const float var = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
-    const float rstd = rsqrtf(var * (1.0f / kCz) + a.eps);
-    const float2 rstd2 = make_float2(rstd, rstd);
-
-    // ---- normalise, bias dot products, bf16 A tile (parameters read as float4,
-    // arithmetic on channel pairs)
-    float2 bacc[kHeads] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                           make_float2(0.f, 0.f)};
-    const float4* g4 = reinterpret_cast<const float4*>(s_gamma);
-    const float4* b4 = reinterpret_cast<const float4*>(s_beta);
-    const float4* w4 = reinterpret_cast<const float4*>(s_wb);
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const uint32_t w[4] = {zr[c].x, zr[c].y, zr[c].z, zr[c].w};
-      float2 xv[4];  // channels 8c .. 8c+7 as pairs
-#pragma unroll
-      for (int hq = 0; hq < 2; ++hq) {
-        const float4 gm = g4[2 * c + hq], bt = b4[2 * c + hq];
-        const float2 d0 = __fadd2_rn(chan2(w[2 * hq]), nmu);
-        const float2 d1 = __fadd2_rn(chan2(w[2 * hq + 1]), nmu);
-        xv[2 * hq] = __ffma2_rn(__fmul2_rn(d0, rstd2), make_float2(gm.x, gm.y),
-                                make_float2(bt.x, bt.y));
-        xv[2 * hq + 1] = __ffma2_rn(__fmul2_rn(d1, rstd2), make_float2(gm.z, gm.w),
-                                    make_float2(bt.z, bt.w));
-      }
+      const int cb = hc * 64 + c * 8;  // first channel of this chunk
 #pragma unroll
       for (int h = 0; h < kHeads; ++h) {
-        const float4 wa = w4[(h * kCz) / 4 + 2 * c], wb = w4[(h * kCz) / 4 + 2 * c + 1];
-        float2 acc2 = bacc[h];
-        acc2 = __ffma2_rn(make_float2(wa.x, wa.y), xv[0], acc2);
-        acc2 = __ffma2_rn(make_float2(wa.z, wa.w), xv[1], acc2);
-        acc2 = __ffma2_rn(make_float2(wb.x, wb.y), xv[2], acc2);
-        acc2 = __ffma2_rn(make_float2(wb.z, wb.w), xv[3], acc2);
-        bacc[h] = acc2;
-      }
-      if (qkvg) {
-        // K-major, 128 B swizzle: row gt, 16-byte chunk (c % 8) of K-slab c / 8
-        uint8_t* dst = sA + (c >> 3) * kAAtomBytes + gt * 128 + (((c & 7) ^ (gt & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) =
-            make_uint4(pack_bf16x2(xv[0].x, xv[0].y), pack_bf16x2(xv[1].x, xv[1].y),
-                       pack_bf16x2(xv[2].x, xv[2].y), pack_bf16x2(xv[3].x, xv[3].y));
+        const float4 wa = w4[(h * kCz + cb) / 4], wb = w4[(h * kCz + cb) / 4 + 1];
+        float2 acc2 = sb[h];
+        acc2 = __ffma2_rn(make_float2(wa.x, wa.y), d[0], acc2);
+        acc2 = __ffma2_rn(make_float2(wa.z, wa.w), d[1], acc2);
+        acc2 = __ffma2_rn(make_float2(wb.x, wb.y), d[2], acc2);
+        acc2 = __ffma2_rn(make_float2(wb.z, wb.w), d[3], acc2);
+        sb[h] = acc2;
       }
     }
-    if (a.write_bias) {
-      const bool key_valid = jv && (a.mask == nullptr || a.mask[j] != 0);
-      if (j < a.ld_bias) {
+    float part[kPartials];
+    part[0] = (s1[0].x + s1[0].y) + (s1[1].x + s1[1].y);
+    part[1] = (s2[0].x + s2[0].y) + (s2[1].x + s2[1].y);
 #pragma unroll
-        for (int h = 0; h < kHeads; ++h)
-          a.bias[(static_cast<long long>(h) * a.bias_rows + (i - a.bias_row0)) * a.ld_bias + j] =
-              __float2bfloat16_rn(key_valid ? bacc[h].x + bacc[h].y : kMaskedLogit);
+    for (int h = 0; h < kHeads; ++h) part[2 + h] = sb[h].x + sb[h].y;
+    // ---- exchange with the other thread of the pair; both sum half 0 + half 1
+#pragma unroll
+    for (int k = 0; k < kPartials; ++k) xch[(hc * kPartials + k) * kTileM + p] = part[k];
+    named_barrier_sync(bar_id, kGroupThreads);
+    float tot[kPartials];
+#pragma unroll
+    for (int k = 0; k < kPartials; ++k) {
+      const float other = xch[((hc ^ 1) * kPartials + k) * kTileM + p];
+      tot[k] = hc == 0 ? part[k] + other : other + part[k];
+    }
+    const float md = tot[0] * (1.0f / kCz);            // mean - K
+    const float var = fmaxf(tot[1] * (1.0f / kCz) - md * md, 0.f);
+    const float rstd = rsqrtf(var + a.eps);
+    if (a.write_bias && j < a.ld_bias) {
+      // heads 2 hc and 2 hc + 1: rstd (S_h - (mean - K) sum_c Wb gamma) + Wb . beta
+      const bool key_valid = jv && (a.mask == nullptr || a.mask[j] != 0);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int h = 2 * hc + hh;
+        const float b = fmaf(fmaf(-md, s_wsum[h], tot[2 + h]), rstd, s_wbeta[h]);
+        a.bias[(static_cast<long long>(h) * a.bias_rows + (i - a.bias_row0)) * a.ld_bias + j] =
+            __float2bfloat16_rn(key_valid ? b : kMaskedLogit);
       }
     }
     if (!qkvg) {
-      // bias only: the buffer is free once every thread of the group has read it
+      // bias only: the buffer (and the exchange area) is free once every
+      // thread of the group has read them
       named_barrier_sync(bar_id, kGroupThreads);
       if (mma_thread && tile + stride < ntiles) {
         issue_z(tile + stride);
         z_pending = true;
       }
       continue;
+    }
+
+    // ---- normalise this thread's 64 channels into the A operand, in place
+    {
+      const float mu = K + md;
+      const float2 nmu = make_float2(-mu, -mu), rstd2 = make_float2(rstd, rstd);
+      const float4* g4 = reinterpret_cast<const float4*>(s_gamma + hc * 64);
+      const float4* b4 = reinterpret_cast<const float4*>(s_beta + hc * 64);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        // read again rather than held across the exchange (register pressure)
+        const uint4 zc = *reinterpret_cast<const uint4*>(row + ((c ^ (p & 7)) << 4));
+        const uint32_t w[4] = {zc.x, zc.y, zc.z, zc.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int hq = 0; hq < 2; ++hq) {
+          const float4 gm = g4[2 * c + hq], bt = b4[2 * c + hq];
+          const float2 d0 = __fadd2_rn(chan2(w[2 * hq]), nmu);
+          const float2 d1 = __fadd2_rn(chan2(w[2 * hq + 1]), nmu);
+          const float2 x0 = __ffma2_rn(__fmul2_rn(d0, rstd2), make_float2(gm.x, gm.y),
+                                       make_float2(bt.x, bt.y));
+          const float2 x1 = __ffma2_rn(__fmul2_rn(d1, rstd2), make_float2(gm.z, gm.w),
+                                       make_float2(bt.z, bt.w));
+          o[2 * hq] = pack_bf16x2(x0.x, x0.y);
+          o[2 * hq + 1] = pack_bf16x2(x1.x, x1.y);
+        }
+        *reinterpret_cast<uint4*>(row + ((c ^ (p & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
     }
 
     fence_proxy_async_smem();
@@ -279,21 +332,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         z_pending = true;
       }
 
-      // ---- epilogue: TMEM lane gt -> two of q, k, v, g of pair j.  Each 32-column
-      // chunk (one head of one output) of the warp's 32 pairs is 32 rows of 64 B,
-      // contiguous in the head-major output: the warp stages it in shared memory
-      // and writes it back with 512-byte coalesced stores.
-      const int jw0 = static_cast<int>(tile % jtiles) * kTileM + (warp & 3) * 32;
-      uint8_t* stg = smem + kSmemStg + warp * kStgBytes;
+      // ---- epilogue: output part = 2 half + hc of pair j, one 32-column chunk
+      // (one head) at a time: the pair's 64-byte row of that head, written with
+      // two 32-byte stores
+      const int part = half * 2 + hc;
+      const uint32_t col0 = tmem + lane_base + hc * 128;
+      __nv_bfloat16* out = part == 0 ? a.Q : part == 1 ? a.K : part == 2 ? a.V : a.G;
       uint32_t v[32], vn[32];
-      tmem_ld32(tmem + lane_base, vn);
+      tmem_ld32(col0, vn);
 #pragma unroll 1
-      for (int cc = 0; cc < 8; ++cc) {
+      for (int h = 0; h < kHeads; ++h) {
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = vn[e];
-        if (cc + 1 < 8) tmem_ld32(tmem + lane_base + (cc + 1) * 32, vn);  // overlap the next load
-        const int part = half * 2 + (cc >> 2), h = cc & 3;
+        if (h + 1 < kHeads) tmem_ld32(col0 + (h + 1) * 32, vn);  // overlap the next load
         uint32_t pk[16];
         if (part < 3) {
           const float sc = part == 0 ? a.q_scale : 1.0f;
@@ -316,24 +368,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          fmaf(0.5f, tanh_approx(0.5f * t3), 0.5f));
           }
         }
-        // The staging buffer is the 64-byte-swizzled image of a 32 x 32 bf16 TMA
-        // box (row = lane, 16-byte chunk q at position q ^ ((lane / 2) % 4), which
-        // is also conflict-free); lane 0 stores it with one TMA store, which
-        // clips the rows past N.  The previous chunk's store must have read the
-        // buffer before it is rewritten.
-        const int lane = gt & 31;
-        if (lane == 0) bulk_wait_read_all();
-        __syncwarp();
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          *reinterpret_cast<uint4*>(stg + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) =
-              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          const CUtensorMap* m = part == 0 ? &map_q : part == 1 ? &map_k : part == 2 ? &map_v : &map_g;
-          tma_store_3d(m, stg, 0, jw0, r * kHeads + h);
-          bulk_commit();
+        if (jv) {
+          uint32_t* dst = reinterpret_cast<uint32_t*>(
+              out + ((static_cast<long long>(r) * kHeads + h) * a.N + j) * kD);
+          st_global_v8(dst, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+          st_global_v8(dst + 8, pk[8], pk[9], pk[10], pk[11], pk[12], pk[13], pk[14], pk[15]);
         }
       }
       tc_fence_before();
@@ -346,8 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // ---- teardown: no bulk copy may still be reading or writing this CTA's smem
-  if ((gt & 31) == 0) bulk_wait_all();
+  // ---- teardown: no copy may still be writing this CTA's smem
   if (tid == 0 && qkvg && !w_ready) {
     if (!mbar_wait(w_bar, 0, nullptr)) report_status(a.status, kStatusTimeout);
   }

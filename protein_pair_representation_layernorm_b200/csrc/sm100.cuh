@@ -136,6 +136,15 @@ __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// 32-byte store to global memory (a whole sector); p must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* p, uint32_t a0, uint32_t a1, uint32_t a2,
+                                             uint32_t a3, uint32_t a4, uint32_t a5, uint32_t a6,
+                                             uint32_t a7) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a0), "r"(a1),
+               "r"(a2), "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+               : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -309,6 +318,18 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   const int a = max(__float_as_int(p.x) + (__float_as_int(t.x) << 23), 0);
   const int b = max(__float_as_int(p.y) + (__float_as_int(t.y) << 23), 0);
   return make_float2(__int_as_float(a), __int_as_float(b));
+}
+
+// (lo, hi) = (bf16 low half of w + s.x, bf16 high half of w + s.y) in fp32, one
+// mixed-precision add per value (the bf16 operand widens exactly, so this equals
+// widening it first and adding in fp32).
+__device__ __forceinline__ float2 add_bf16x2_f32x2(uint32_t w, float2 s) {
+  float2 r;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %3;\n\tadd.rn.f32.bf16 %1, hi, %4;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "r"(w), "f"(s.x), "f"(s.y));
+  return r;
 }
 
 __device__ __forceinline__ float tanh_approx(float x) {

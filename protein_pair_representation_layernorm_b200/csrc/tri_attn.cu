@@ -509,18 +509,8 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
     if (!make_map_3d(&mz, Zb, kCz, N, zrows, kCz * 2, static_cast<uint64_t>(N) * kCz * 2, 64, zb1,
                      CU_TENSOR_MAP_SWIZZLE_128B, zb2))
       return cudaErrorInvalidValue;
-    // q, k, v, g outputs ([rows][H][N][d] bf16): 32 x 32 boxes, 64 B swizzle (the
-    // kernel's per-warp staging layout); a bias-only pass never stores through them
-    CUtensorMap mo[4];
-    void* outs[4] = {a.Q, a.K, a.V, a.G};
-    const uint64_t rh = static_cast<uint64_t>(wq ? nrows : 1) * kHeads;
-    for (int m = 0; m < 4; ++m)
-      if (!make_map_3d(&mo[m], outs[m], kD, N, rh, kD * 2, static_cast<uint64_t>(N) * kD * 2, kD,
-                       32, CU_TENSOR_MAP_SWIZZLE_64B))
-        return cudaErrorInvalidValue;
     Timer tm(h, st, timed, 0);
-    tri::plp::pair_ln_proj<<<grid, tri::plp::kThreads, tri::plp::kSmemBytes, st>>>(
-        mz, mo[0], mo[1], mo[2], mo[3], a);
+    tri::plp::pair_ln_proj<<<grid, tri::plp::kThreads, tri::plp::kSmemBytes, st>>>(mz, a);
     return cudaGetLastError();
   };
   if (slab && slab->phase == 0) {  // the slab's bias rows only

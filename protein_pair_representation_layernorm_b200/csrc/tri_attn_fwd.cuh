@@ -321,9 +321,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
+          // s + b with the bf16 bias as the operand of a mixed-precision add (no
+          // separate widening of the bias)
           float2& xe = x[half * 16 + e];
-          xe = __fadd2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
-                          make_float2(bf16lo_to_f32(bw[e]), bf16hi_to_f32(bw[e])));
+          xe = add_bf16x2_f32x2(bw[e],
+                                make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])));
           mx[e & 3] = fmax3(mx[e & 3], xe.x, xe.y);
         }
       }
