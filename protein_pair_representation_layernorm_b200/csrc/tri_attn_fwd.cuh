@@ -38,10 +38,11 @@
 //
 // Exponentials: 16 per clock per SM on the special-function unit, one per
 // score, which makes that unit the kernel's ceiling at head width 32; one
-// pair in eight is evaluated on the FMA pipe instead (exp2_poly2: Cody-Waite
+// pair in four is evaluated on the FMA pipe instead (exp2_poly2: Cody-Waite
 // reduction and a degree-3 polynomial fitted to 7.5e-5 relative error, far
-// below the bf16 rounding of P), which measured ~1% faster than none, 1/4,
-// 1/10 or 1/16.
+// below the bf16 rounding of P): with the bias added by a mixed-precision add
+// (one instruction per score) that share measured fastest (5.21 ms at
+// N = 1536 against 5.34 with one pair in eight and 5.37 with none).
 //
 // Online softmax per (row, query): the running offset m is raised only when a
 // tile's maximum exceeds it by more than kTau (log2 units), so O is rarely
@@ -367,9 +368,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q = 0; q < 8; ++q) {
           const int e = quarter * 8 + q;
           const float2 dlt = __fadd2_rn(x[e], neg_m);
-          // the last pair of every 8 on the FMA pipe (exp2_poly2), the rest on
+          // the last pair of every 4 on the FMA pipe (exp2_poly2), the rest on
           // the special-function unit, which is the busiest unit of the kernel
-          const float2 p = (e % 8 == 7) ? exp2_poly2(dlt)
+          const float2 p = (e % 4 == 3) ? exp2_poly2(dlt)
                                         : make_float2(ex2_approx(dlt.x), ex2_approx(dlt.y));
           acc[e & 1] = __fadd2_rn(acc[e & 1], p);
           pk[q] = pack_bf16x2(p.x, p.y);
