@@ -50,10 +50,13 @@ EX2_SHARE = 0.75         # the attention kernel evaluates one exponential pair i
 NUM_SMS = 148
 SM_MAX_MHZ = 1965.0
 
-# DRAM bytes per tri_attn_fwd launch (starting node, N = 1536) from one ncu
-# capture of this kernel source, valid only for the source with this hash;
+# DRAM bytes per tri_attn_fwd launch at N = 1536, from one ncu capture of this
+# kernel source at N = 768 (ending node; 457.8 MB read + 133.9 MB written)
+# scaled by the ratio of pairs (4): Q, K, V read once, O written once, and the
+# logit bias all grow with N^2.  Valid only for the source with this hash;
 # otherwise reported as null.
-TRAFFIC = {"tri_attn_fwd.cuh": "f9c788dbdbff8c0d", "bytes_per_launch": 1.832449e9 + 0.584904e9}
+TRAFFIC = {"tri_attn_fwd.cuh": "d277a929470fd6db", "bytes_per_launch": 4 * (457.800192e6 + 133.886464e6),
+           "measured_at": "N=768, scaled x4 to N=1536"}
 
 
 def parse():
@@ -352,6 +355,8 @@ def run_ours(args, world, rank, local):
         "roofline": {"kernel": "tri_attn_fwd", "bound": "tensor", "achieved": attn_tf,
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": attn_tf / peak_tf,
                      "peak_source": f"{peak_src} bf16_tflops (burst)", "traffic": traffic,
+                     "traffic_source": (f"ncu dram__bytes_read.sum + dram__bytes_write.sum, "
+                                        f"{TRAFFIC['measured_at']}") if traffic else None,
                      "algorithmic_flops_per_launch": flops_attn,
                      "launch_ms": attn_ms,
                      # the unit that caps the kernel at head width 32: one exp2 per
