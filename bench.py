@@ -308,8 +308,10 @@ def run_ours(args, world, rank, local):
     pairs = N * N
     proj_ms = kms[0] / max(kn[0], 1)
     gate_ms = kms[2] / max(kn[2], 1)
-    proj_bytes = pairs * (256 + 1024) + 4 * N * ((N + 63) // 64 * 64) * 2
-    gate_bytes = pairs * (768 + 256)
+    # pair_ln_proj reads z (256 B a pair) and writes q, k, v (768 B) and the bias;
+    # gate_out reads o and z (512 B) and writes out (256 B)
+    proj_bytes = pairs * (256 + 768) + 4 * N * ((N + 63) // 64 * 64) * 2
+    gate_bytes = pairs * (512 + 256)
     traffic = None
     if TRAFFIC["tri_attn_fwd.cuh"] == src_hash("tri_attn_fwd.cuh"):
         traffic = TRAFFIC["bytes_per_launch"]

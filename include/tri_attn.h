@@ -161,7 +161,9 @@ size_t tri_attn_workspace_bytes(tri_attn_dtype dtype, int N);
  * -inf for F32 handles and the finite -3e38 for BF16 handles, which keeps the
  * sums it enters finite and still gives those keys probability exactly 0;
  * q already scaled by log2(e)/sqrt(d)).  Element type: bf16 for a BF16
- * handle, fp32 for F32.  Any output pointer may be NULL. */
+ * handle, fp32 for F32.  A BF16 handle keeps no gate tensor (gate_out
+ * recomputes the gate from LayerNorm(z)), so *g is set to NULL for it.  Any
+ * output pointer may be NULL. */
 int tri_attn_debug_workspace(tri_attn_handle *h, void **q, void **k, void **v, void **g,
                              void **bias, void **o, int *ld_bias, int *rows);
 
@@ -221,7 +223,7 @@ int tri_attn_rows_forward(tri_attn_handle *h, const void *Z_rows, int N, int row
  * of 32 MiB inside this library; every GPU that loads the library holds it
  * until the process exits.  Rows are processed in chunks that fit the array.
  * Sizes it cannot hold (the whole logit bias plus one three-row chunk must fit,
- * which allows N up to 1792) return TRI_ATTN_ERR_UNSUPPORTED before anything
+ * which allows N up to 1856) return TRI_ATTN_ERR_UNSUPPORTED before anything
  * is launched.  The first call on a device also looks up the array's
  * device address (cudaGetSymbolAddress); make that first call before any stream
  * capture.  All calls share the one array, which keeps the last call's contents

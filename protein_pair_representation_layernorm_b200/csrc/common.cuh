@@ -58,10 +58,10 @@ struct ProjArgs {
   const uint8_t* mask;
   int N, orient, row0, rows;
   int write_qkvg, write_bias;
-  const uint8_t* w_img;  // W_qkvg as the shared-memory image of the MMA B operand
-  const float *w_b, *gamma, *beta, *b_g;  // w_b pre-scaled by log2(e)
+  const uint8_t* w_img;  // [Wq; Wk; Wv] as the shared-memory image of the MMA B operand
+  const float *w_b, *gamma, *beta;  // w_b pre-scaled by log2(e)
   float eps, q_scale;
-  __nv_bfloat16 *Q, *K, *V, *G, *bias;
+  __nv_bfloat16 *Q, *K, *V, *bias;
   int ld_bias;
   // Z holds problem rows z_row0.. (a row slab; 0 for the whole tensor), and the
   // bias buffer holds, per head, bias_rows problem rows starting at bias_row0
@@ -78,9 +78,11 @@ struct AttnArgs {
 };
 
 struct GateArgs {
-  const __nv_bfloat16 *Z, *O, *G;
+  const __nv_bfloat16 *Z, *O;
   const uint8_t* wo_img;  // W_o as the shared-memory image of the MMA B operand
-  const float* b_o;
+  const uint8_t* wg_img;  // W_g likewise: the gate is recomputed from LayerNorm(z)
+  const float *b_o, *b_g, *gamma, *beta;
+  float eps;
   __nv_bfloat16* out;
   int N, orient, row0, rows;
   int z_row0;  // Z and out hold problem rows z_row0.. (a row slab; 0 for the whole tensor)

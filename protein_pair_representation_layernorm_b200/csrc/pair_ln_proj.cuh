@@ -1,4 +1,4 @@
-// pair_ln_proj.cuh — LayerNorm + fused Q/K/V/gate projection (tcgen05) + logit
+// pair_ln_proj.cuh — LayerNorm + fused Q/K/V projection (tcgen05) + logit
 // bias, bf16 pair representation.
 //
 // Persistent CTAs of two independent groups of 8 warps.  Each group walks its
@@ -20,19 +20,21 @@
 //      kMaskedLogit at masked keys and at the padding columns j >= N,
 //   4. writes its normalised channels as bf16 back in place, which makes the
 //      buffer the A operand.
-// One thread of the group then issues the projection D = X W^T in two halves of
-// N = 256 (q|k, then v|g), W = [Wq; Wk; Wv; Wg] resident in shared memory for the
-// whole kernel, each half accumulating in fp32 in the group's 256 TMEM columns;
-// the next tile's TMA is issued as soon as the second half has consumed the
-// buffer.  In the epilogue of a half the two threads of a pair take one output
-// each (q or k, v or g): the thread reads its TMEM lane, scales q by
-// log2(e)/sqrt(d), forms sigmoid(g + bg), and writes the pair's 64-byte row of
-// each head of the head-major output ([rows][H][N][d], bf16) with two 32-byte
-// stores straight from registers (a warp's 32 pairs fill a contiguous 2 KB
-// block).  While one group runs its MMAs the other normalises or stores, so the
-// tensor core, the ALUs and HBM overlap.
+// One thread of the group then issues the projection D = X W^T in two halves,
+// N = 256 (q|k) and then N = 128 (v), W = [Wq; Wk; Wv] resident in shared
+// memory for the whole kernel, each half accumulating in fp32 in the group's
+// 256 TMEM columns; the next tile's TMA is issued as soon as the second half
+// has consumed the buffer.  In the epilogue of the q|k half the two threads of
+// a pair take q (scaled by log2(e)/sqrt(d)) and k, in that of the v half two
+// heads of v each: the thread reads its TMEM lane and writes the pair's 64-byte
+// row of each head of the head-major output ([rows][H][N][d], bf16) with two
+// 32-byte stores straight from registers (a warp's 32 pairs fill a contiguous
+// 2 KB block).  The gate is not produced here: gate_out recomputes it from
+// LayerNorm(z), which it reads anyway, so it never goes through memory.  While
+// one group runs its MMAs the other normalises or stores, so the tensor core,
+// the ALUs and HBM overlap.
 //
-// This is the HBM-bound step: per pair it reads 256 B and writes 1 KB + 8 B.
+// This is the HBM-bound step: per pair it reads 256 B and writes 768 B + 8 B.
 #pragma once
 
 #include "common.cuh"
@@ -45,16 +47,16 @@ constexpr int kGroupThreads = 256;                   // two threads per pair
 constexpr int kGroupsPerCta = 2;
 constexpr int kThreads = kGroupThreads * kGroupsPerCta;
 constexpr int kTileM = 128;
-constexpr int kNOut = 4 * kHD;                       // q | k | v | g
-constexpr uint32_t kWImgBytes = kNOut * kCz * 2;     // 131072
+constexpr int kNOut = 3 * kHD;                       // q | k | v
+constexpr uint32_t kWImgBytes = kNOut * kCz * 2;     // 98304
 constexpr uint32_t kWAtomBytes = kNOut * 128;        // one 64-element K slab of W
 constexpr uint32_t kATileBytes = kTileM * kCz * 2;   // 32768
 constexpr uint32_t kAAtomBytes = kTileM * 128;       // 16384: one 64-channel box
 constexpr uint32_t kSmemW = 0;
 constexpr uint32_t kSmemA = kWImgBytes;                                  // + grp * kATileBytes
 constexpr uint32_t kSmemPar = kSmemA + kGroupsPerCta * kATileBytes;     // fp32 params
-// w_b * gamma [H][c_z], gamma, beta, b_g, then per head sum_c w_b gamma and w_b . beta
-constexpr uint32_t kParFloats = kHeads * kCz + 3 * kCz + 2 * kHeads;
+// w_b * gamma [H][c_z], gamma, beta, then per head sum_c w_b gamma and w_b . beta
+constexpr uint32_t kParFloats = kHeads * kCz + 2 * kCz + 2 * kHeads;
 constexpr int kPartials = 2 + kHeads;                // sum, sum of squares, 4 bias dots
 constexpr uint32_t kSmemXch = kSmemPar + ((kParFloats * 4 + 15) / 16) * 16;
 // [group][channel half][partial][pair]
@@ -72,8 +74,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* s_wbg = reinterpret_cast<float*>(smem + kSmemPar);  // w_b[h][c] * gamma[c]
   float* s_gamma = s_wbg + kHeads * kCz;
   float* s_beta = s_gamma + kCz;
-  float* s_bg = s_beta + kCz;
-  float* s_wsum = s_bg + kCz;        // [h]: sum_c w_b[h][c] gamma[c]
+  float* s_wsum = s_beta + kCz;      // [h]: sum_c w_b[h][c] gamma[c]
   float* s_wbeta = s_wsum + kHeads;  // [h]: sum_c w_b[h][c] beta[c]
   float* s_xch = reinterpret_cast<float*>(smem + kSmemXch);
   uint64_t* w_bar = reinterpret_cast<uint64_t*>(smem + kSmemBar);
@@ -97,7 +98,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int idx = tid; idx < kCz; idx += kThreads) {
     s_gamma[idx] = a.gamma[idx];
     s_beta[idx] = a.beta[idx];
-    s_bg[idx] = a.b_g[idx];
   }
   if (warp < kHeads) {  // per-head constants of the bias: one warp per head
     float sw = 0.f, sb = 0.f;
@@ -144,7 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long stride = static_cast<long long>(gridDim.x) * kGroupsPerCta;
   const uint32_t sA_u32 = smem_u32(sA), sW_u32 = smem_u32(smem + kSmemW);
   const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-  constexpr uint32_t kIdesc = idesc_bf16_f32(128, 256, false);
+  constexpr uint32_t kIdesc = idesc_bf16_f32(128, 256, false);   // q | k
+  constexpr uint32_t kIdescV = idesc_bf16_f32(128, 128, false);  // v
   uint32_t mma_phase = 0;
   bool w_ready = false;
   const bool mma_thread = gt == 0;
@@ -297,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
 #pragma unroll 1
     for (int half = 0; half < 2; ++half) {
-      // ---- MMA: D[128 x 256] = X W[half*256 .. half*256+255]^T
+      // ---- MMA: D = X W_half^T, W_half = rows 0..255 of W (q|k) or 256..383 (v)
       if (mma_thread) {
         bool ready = true;
         if (!w_ready) {
@@ -312,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t bd = smem_desc(
                 sW_u32 + (kk >> 2) * kWAtomBytes + half * 256 * 128 + (kk & 3) * 32, 1024,
                 kSwizzle128B);
-            mma_ss(tmem, ad, bd, kIdesc, kk > 0 ? 1u : 0u);
+            mma_ss(tmem, ad, bd, half == 0 ? kIdesc : kIdescV, kk > 0 ? 1u : 0u);
           }
           mma_commit(&mma_bar[grp]);
         } else {
@@ -332,42 +333,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         z_pending = true;
       }
 
-      // ---- epilogue: output part = 2 half + hc of pair j, one 32-column chunk
-      // (one head) at a time: the pair's 64-byte row of that head, written with
-      // two 32-byte stores
-      const int part = half * 2 + hc;
-      const uint32_t col0 = tmem + lane_base + hc * 128;
-      __nv_bfloat16* out = part == 0 ? a.Q : part == 1 ? a.K : part == 2 ? a.V : a.G;
+      // ---- epilogue, one 32-column chunk (one head) at a time: after the q|k
+      // half the two threads of a pair take q and k (4 heads each), after the v
+      // half two heads of v each; a chunk is the pair's 64-byte row of that head,
+      // written with two 32-byte stores
+      const int nchunks = half == 0 ? kHeads : 2;
+      const uint32_t col0 = tmem + lane_base + (half == 0 ? hc * 128 : hc * 64);
+      __nv_bfloat16* out = half == 0 ? (hc == 0 ? a.Q : a.K) : a.V;
+      const float sc = half == 0 && hc == 0 ? a.q_scale : 1.0f;
       uint32_t v[32], vn[32];
       tmem_ld32(col0, vn);
 #pragma unroll 1
-      for (int h = 0; h < kHeads; ++h) {
+      for (int cc = 0; cc < nchunks; ++cc) {
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = vn[e];
-        if (h + 1 < kHeads) tmem_ld32(col0 + (h + 1) * 32, vn);  // overlap the next load
+        if (cc + 1 < nchunks) tmem_ld32(col0 + (cc + 1) * 32, vn);  // overlap the next load
+        const int h = half == 0 ? cc : 2 * hc + cc;
         uint32_t pk[16];
-        if (part < 3) {
-          const float sc = part == 0 ? a.q_scale : 1.0f;
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
-        } else {
-          // sigmoid(t) = 1/2 + tanh(t/2)/2: one special-function op per value
-          const float4* bg4 = reinterpret_cast<const float4*>(s_bg + h * kD);
-#pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 bb = bg4[e4];
-            const float t0 = __uint_as_float(v[4 * e4]) + bb.x;
-            const float t1 = __uint_as_float(v[4 * e4 + 1]) + bb.y;
-            const float t2 = __uint_as_float(v[4 * e4 + 2]) + bb.z;
-            const float t3 = __uint_as_float(v[4 * e4 + 3]) + bb.w;
-            pk[2 * e4] = pack_bf16x2(fmaf(0.5f, tanh_approx(0.5f * t0), 0.5f),
-                                     fmaf(0.5f, tanh_approx(0.5f * t1), 0.5f));
-            pk[2 * e4 + 1] = pack_bf16x2(fmaf(0.5f, tanh_approx(0.5f * t2), 0.5f),
-                                         fmaf(0.5f, tanh_approx(0.5f * t3), 0.5f));
-          }
-        }
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
         if (jv) {
           uint32_t* dst = reinterpret_cast<uint32_t*>(
               out + ((static_cast<long long>(r) * kHeads + h) * a.N + j) * kD);

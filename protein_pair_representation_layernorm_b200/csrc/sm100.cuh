@@ -348,6 +348,24 @@ __device__ __forceinline__ float bf16hi_to_f32(uint32_t v) {
   return __uint_as_float(v & 0xFFFF0000u);
 }
 
+// A value the compiler cannot see through: re-deriving a shared-memory address
+// with it inside a loop keeps loads of loop-invariant parameters in the loop,
+// instead of hoisted into registers for its whole length.
+__device__ __forceinline__ uint32_t opaque_u32(uint32_t x) {
+  asm volatile("" : "+r"(x));
+  return x;
+}
+
+// 16-byte load from shared memory (a 16-byte aligned shared-window address).
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+      : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+      : "r"(addr)
+      : "memory");
+  return v;
+}
+
 // Named barrier for a subset of the CTA's warps.
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

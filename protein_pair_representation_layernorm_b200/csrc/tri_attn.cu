@@ -202,7 +202,8 @@ struct tri_attn_handle {
   float eps = 1e-5f;
   float q_scale = 0.f;
   // packed weights (device)
-  void* w_qkvg = nullptr;  // bf16: MMA B image (128 KB); f32: [512][128]
+  void* w_qkvg = nullptr;  // bf16: [Wq; Wk; Wv] MMA B image (96 KB); f32: [Wq; Wk; Wv; Wg] [512][128]
+  void* w_g = nullptr;     // bf16: Wg MMA B image (32 KB), for the gate recomputed in gate_out
   void* w_o = nullptr;     // bf16: MMA B image (32 KB);  f32: [128][128]
   float* w_b = nullptr;    // [H][c_z], times log2(e)
   float* gamma = nullptr;
@@ -243,24 +244,30 @@ size_t bias_bytes(tri_attn_dtype dt, int N) {
   return align_up(static_cast<size_t>(kHeads) * N * ld_bias_for(N) * esize(dt), 256);
 }
 
+// Per-pair intermediates in the workspace: Q, K, V, O (H*d each), and for fp32
+// handles also G; bf16 handles recompute the gate in gate_out from LayerNorm(z),
+// so G never reaches memory.
+int pair_buffers(tri_attn_dtype dt) { return dt == TRI_ATTN_F32 ? 5 : 4; }
+
 size_t row_bytes(tri_attn_dtype dt, int N) {
-  // Q, K, V, O: H*d per pair; G: H*d per pair
-  return static_cast<size_t>(N) * 5 * kHD * esize(dt);
+  return static_cast<size_t>(N) * pair_buffers(dt) * kHD * esize(dt);
 }
 
 struct Layout {
   size_t q, k, v, g, o, bias, total;
+  bool has_g;
 };
 
 Layout layout_for(tri_attn_dtype dt, int N, int rows) {
   Layout L{};
   const size_t per = align_up(static_cast<size_t>(rows) * N * kHD * esize(dt), 256);
+  L.has_g = pair_buffers(dt) == 5;
   L.q = 0;
   L.k = per;
   L.v = 2 * per;
-  L.g = 3 * per;
-  L.o = 4 * per;
-  L.bias = 5 * per;
+  L.g = L.has_g ? 3 * per : 0;
+  L.o = (L.has_g ? 4 : 3) * per;
+  L.bias = L.o + per;
   L.total = L.bias + bias_bytes(dt, N);
   return L;
 }
@@ -372,7 +379,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
   h->q = ws + L.q;
   h->k = ws + L.k;
   h->v = ws + L.v;
-  h->g = ws + L.g;
+  h->g = L.has_g ? ws + L.g : nullptr;
   h->o = ws + L.o;
   h->bias = (slab && slab->phase == 1) ? slab->bias_io : static_cast<void*>(ws + L.bias);
   h->ld_bias = ld;
@@ -471,7 +478,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
   bf16* outb = static_cast<bf16*>(out);
   const int jtiles = (N + 127) / 128;
   auto proj = [&](int row0, int nrows, int wq, int wb, int out_off = 0) {
-    const size_t off = static_cast<size_t>(out_off) * kHeads * N * kD;  // rows into Q/K/V/G
+    const size_t off = static_cast<size_t>(out_off) * kHeads * N * kD;  // rows into Q/K/V
     tri::ProjArgs a{};
     a.Z = Zb;
     a.mask = mask;
@@ -485,13 +492,11 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
     a.w_b = h->w_b;
     a.gamma = h->gamma;
     a.beta = h->beta;
-    a.b_g = h->b_g;
     a.eps = h->eps;
     a.q_scale = h->q_scale;
     a.Q = static_cast<bf16*>(h->q) + off;
     a.K = static_cast<bf16*>(h->k) + off;
     a.V = static_cast<bf16*>(h->v) + off;
-    a.G = static_cast<bf16*>(h->g) + off;
     a.bias = static_cast<bf16*>(slab && slab->phase == 0 ? slab->bias_io : h->bias);
     a.ld_bias = ld;
     a.z_row0 = rbeg;
@@ -559,15 +564,13 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
       CUDA_TRY(cudaGetLastError());
     }
     {
-      // o, g: this chunk's workspace (head-major); z, out: the pair tensor, boxes of 128 pairs
+      // o: this chunk's workspace (head-major); z, out: the pair tensor, boxes of 128 pairs
       // along j (starting node) or, through the swapped view, along the rows of Z
-      CUtensorMap mo, mg, mz, mout;
+      CUtensorMap mo, mz, mout;
       const uint64_t rowb = static_cast<uint64_t>(N) * kCz * 2;
       const uint32_t zb1 = orient == 0 ? 128u : 1u, zb2 = orient == 0 ? 1u : 128u;
       bool okm =
           make_map_3d(&mo, h->o, kD, N, static_cast<uint64_t>(nr) * kHeads, kD * 2,
-                      static_cast<uint64_t>(N) * kD * 2, kD, 128, CU_TENSOR_MAP_SWIZZLE_64B) &&
-          make_map_3d(&mg, h->g, kD, N, static_cast<uint64_t>(nr) * kHeads, kD * 2,
                       static_cast<uint64_t>(N) * kD * 2, kD, 128, CU_TENSOR_MAP_SWIZZLE_64B) &&
           make_map_3d(&mz, Zb, kCz, N, zrows, kCz * 2, rowb, 64, zb1, CU_TENSOR_MAP_SWIZZLE_128B,
                       zb2) &&
@@ -577,9 +580,13 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
       tri::GateArgs a{};
       a.Z = Zb;
       a.O = static_cast<const bf16*>(h->o);
-      a.G = static_cast<const bf16*>(h->g);
       a.wo_img = static_cast<const uint8_t*>(h->w_o);
+      a.wg_img = static_cast<const uint8_t*>(h->w_g);
       a.b_o = h->b_o;
+      a.b_g = h->b_g;
+      a.gamma = h->gamma;
+      a.beta = h->beta;
+      a.eps = h->eps;
       a.out = outb;
       a.N = N;
       a.orient = orient;
@@ -591,8 +598,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
       const long long ntiles = static_cast<long long>(nr) * jtiles;
       const unsigned grid = static_cast<unsigned>(std::min<long long>(ntiles, h->num_sms));
       Timer tm(h, st, timed, 2);
-      tri::gout::gate_out<<<grid, tri::gout::kThreads, tri::gout::kSmemBytes, st>>>(mo, mg, mz,
-                                                                                   mout, a);
+      tri::gout::gate_out<<<grid, tri::gout::kThreads, tri::gout::kSmemBytes, st>>>(mo, mz, mout, a);
       CUDA_TRY(cudaGetLastError());
     }
     if (hook && hook->after) {
@@ -694,18 +700,22 @@ int tri_attn_create(const tri_attn_params* p, tri_attn_handle** out) {
   for (float& x : wb) x *= tri::kLog2e;
 
   if (dt == TRI_ATTN_BF16) {
-    // [Wq; Wk; Wv; Wg] as 512 K-major rows, and Wo as 128 K-major rows, both in the
-    // shared-memory image the tcgen05 B operand reads (bf16 bits kept exactly).
-    std::vector<uint16_t> w512(512 * 128), w128(128 * 128), img;
-    const std::vector<float>* parts[4] = {&wq, &wk, &wv, &wg};
-    for (int part = 0; part < 4; ++part)
+    // [Wq; Wk; Wv] as 384 K-major rows, Wg and Wo as 128 K-major rows each, all in
+    // the shared-memory image the tcgen05 B operand reads (bf16 bits kept exactly).
+    std::vector<uint16_t> w384(384 * 128), wg128(128 * 128), w128(128 * 128), img;
+    const std::vector<float>* parts[3] = {&wq, &wk, &wv};
+    for (int part = 0; part < 3; ++part)
       for (int n = 0; n < kHD; ++n)
         for (int c = 0; c < kCz; ++c)
-          w512[(part * kHD + n) * 128 + c] = f32_to_bf16_bits((*parts[part])[n * kCz + c]);
+          w384[(part * kHD + n) * 128 + c] = f32_to_bf16_bits((*parts[part])[n * kCz + c]);
+    for (int n = 0; n < kHD; ++n)
+      for (int c = 0; c < kCz; ++c) wg128[n * 128 + c] = f32_to_bf16_bits(wg[n * kCz + c]);
     for (int n = 0; n < kCz; ++n)
       for (int c = 0; c < kHD; ++c) w128[n * 128 + c] = f32_to_bf16_bits(wo[n * kHD + c]);
-    pack_kmajor_sw128(w512, 512, img);
+    pack_kmajor_sw128(w384, 384, img);
     if ((rc = upload(img, &h->w_qkvg))) return fail(rc);
+    pack_kmajor_sw128(wg128, 128, img);
+    if ((rc = upload(img, &h->w_g))) return fail(rc);
     pack_kmajor_sw128(w128, 128, img);
     if ((rc = upload(img, &h->w_o))) return fail(rc);
   } else {
@@ -977,7 +987,7 @@ int tri_attn_debug_workspace(tri_attn_handle* h, void** q, void** k, void** v, v
 int tri_attn_destroy(tri_attn_handle* h) {
   if (!h) return TRI_ATTN_OK;
   cudaSetDevice(h->device);
-  void* ptrs[] = {h->w_qkvg, h->w_o, h->w_b, h->gamma, h->beta, h->b_g,
+  void* ptrs[] = {h->w_qkvg, h->w_g, h->w_o, h->w_b, h->gamma, h->beta, h->b_g,
                   h->b_o,    h->status, h->ws, h->stage, h->stage_mask};
   for (void* p : ptrs)
     if (p) cudaFree(p);
@@ -1005,8 +1015,9 @@ int tri_attn_destroy(tri_attn_handle* h) {
 namespace {
 
 constexpr size_t kNoallocScratchBytes = size_t(32) << 20;  // 32 MiB per device
-constexpr size_t kNaWImg = 0;                                // 512 x 128 bf16 image
-constexpr size_t kNaWoImg = kNaWImg + 512 * 128 * 2;         // 128 x 128 bf16 image
+constexpr size_t kNaWImg = 0;                                // [Wq; Wk; Wv]: 384 x 128 bf16 image
+constexpr size_t kNaWgImg = kNaWImg + 384 * 128 * 2;         // Wg: 128 x 128 bf16 image
+constexpr size_t kNaWoImg = kNaWgImg + 128 * 128 * 2;        // Wo: 128 x 128 bf16 image
 constexpr size_t kNaWb = kNaWoImg + 128 * 128 * 2;           // fp32 [H][c_z] x log2(e)
 constexpr size_t kNaGamma = kNaWb + kHeads * kCz * 4;
 constexpr size_t kNaBeta = kNaGamma + kCz * 4;
@@ -1038,22 +1049,25 @@ __global__ void pack_weights_noalloc(const bf16* wq, const bf16* wk, const bf16*
                                      const bf16* wg, const bf16* wo, const bf16* wb,
                                      const bf16* gamma, const bf16* beta, const bf16* bg,
                                      const bf16* bo, unsigned char* scratch) {
-  const int n_w = 512 * 128, n_wo = 128 * 128, n_wb = kHeads * kCz;
-  const int total = n_w + n_wo + n_wb + 4 * kCz;
+  const int n_w = 384 * 128, n_wg = 128 * 128, n_wo = 128 * 128, n_wb = kHeads * kCz;
+  const int total = n_w + n_wg + n_wo + n_wb + 4 * kCz;
   for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += gridDim.x * blockDim.x) {
     if (idx < n_w) {
       const int n = idx / 128, k = idx % 128, part = n / kHD, nn = n % kHD;
-      const bf16* src = part == 0 ? wq : part == 1 ? wk : part == 2 ? wv : wg;
-      *reinterpret_cast<bf16*>(scratch + kNaWImg + sw128_offset(512, n, k)) = src[nn * kCz + k];
-    } else if (idx < n_w + n_wo) {
+      const bf16* src = part == 0 ? wq : part == 1 ? wk : wv;
+      *reinterpret_cast<bf16*>(scratch + kNaWImg + sw128_offset(384, n, k)) = src[nn * kCz + k];
+    } else if (idx < n_w + n_wg) {
       const int t = idx - n_w, n = t / 128, k = t % 128;
+      *reinterpret_cast<bf16*>(scratch + kNaWgImg + sw128_offset(128, n, k)) = wg[n * kCz + k];
+    } else if (idx < n_w + n_wg + n_wo) {
+      const int t = idx - n_w - n_wg, n = t / 128, k = t % 128;
       *reinterpret_cast<bf16*>(scratch + kNaWoImg + sw128_offset(128, n, k)) = wo[n * kHD + k];
-    } else if (idx < n_w + n_wo + n_wb) {
-      const int t = idx - n_w - n_wo;
+    } else if (idx < n_w + n_wg + n_wo + n_wb) {
+      const int t = idx - n_w - n_wg - n_wo;
       reinterpret_cast<float*>(scratch + kNaWb)[t] = __bfloat162float(wb[t]) * tri::kLog2e;
     } else {
-      const int t = idx - n_w - n_wo - n_wb, which = t / kCz, c = t % kCz;
+      const int t = idx - n_w - n_wg - n_wo - n_wb, which = t / kCz, c = t % kCz;
       if (which == 0) reinterpret_cast<float*>(scratch + kNaGamma)[c] = __bfloat162float(gamma[c]);
       if (which == 1) reinterpret_cast<float*>(scratch + kNaBeta)[c] = __bfloat162float(beta[c]);
       if (which == 2)
@@ -1133,6 +1147,7 @@ extern "C" int tri_attn_forward_noalloc(const tri_attn_params* p, const void* Z,
   hh.eps = p->ln_eps;
   hh.q_scale = tri::kLog2e / std::sqrt(static_cast<float>(kD));
   hh.w_qkvg = scratch + kNaWImg;
+  hh.w_g = scratch + kNaWgImg;
   hh.w_o = scratch + kNaWoImg;
   hh.w_b = reinterpret_cast<float*>(scratch + kNaWb);
   hh.gamma = reinterpret_cast<float*>(scratch + kNaGamma);

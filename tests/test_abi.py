@@ -37,10 +37,14 @@ def test_workspace_bytes():
     ws = binding.tri_attn_workspace_bytes
     assert ws(binding.TRI_ATTN_BF16, 0) == 0
     assert ws(7, 10) == 0
-    # bf16: q, k, v, g, o (N*N*128 each) + bias H*N*roundup(N,64), 2 bytes per element
-    N = 1536
-    assert ws(binding.TRI_ATTN_BF16, N) >= 5 * N * N * 128 * 2 + 4 * N * N * 2
-    assert ws(binding.TRI_ATTN_F32, N) == 2 * ws(binding.TRI_ATTN_BF16, N)
+    # bf16: q, k, v, o (N*N*128 each; the gate is recomputed, never stored) +
+    # bias H*N*roundup(N,64), 2 bytes per element; fp32: q, k, v, g, o + bias, 4 bytes
+    for N in (1536, 200):
+        ld = -(-N // 64) * 64
+        bias = -(-4 * N * ld * 2 // 256) * 256
+        assert ws(binding.TRI_ATTN_BF16, N) == 4 * N * N * 128 * 2 + bias
+        bias = -(-4 * N * ld * 4 // 256) * 256
+        assert ws(binding.TRI_ATTN_F32, N) == 5 * N * N * 128 * 4 + bias
     assert ws(binding.TRI_ATTN_BF16, 4096) > ws(binding.TRI_ATTN_BF16, 1536)
 
 

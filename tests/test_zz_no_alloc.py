@@ -18,7 +18,7 @@ from protein_pair_representation_layernorm_b200 import binding, workloads
 
 pytestmark = pytest.mark.gpu
 
-MAX_N = 1792  # the largest N whose whole bias plus one three-row chunk fits the 32 MiB array
+MAX_N = 1856  # the largest N whose whole bias plus one three-row chunk fits the 32 MiB array
 
 
 def _params(w: dict) -> binding.tri_attn_params:
@@ -78,8 +78,8 @@ def test_noalloc_matches_handle_entry_point_twice():
 
 
 def test_noalloc_largest_supported_size():
-    """N = 1792 runs (in three-row chunks) and equals the handle path on
-    sampled rows and columns, bit for bit; N = 1793 is rejected before any
+    """N = 1856 runs (in three-row chunks) and equals the handle path on
+    sampled rows and columns, bit for bit; N = 1857 is rejected before any
     launch."""
     N = MAX_N
     inp = workloads.make_inputs(N, "bf16", 63, "random:0.05")
