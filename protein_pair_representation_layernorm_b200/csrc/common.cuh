@@ -79,8 +79,10 @@ struct AttnArgs {
 
 struct GateArgs {
   const __nv_bfloat16 *Z, *O;
-  const uint8_t* wo_img;  // W_o as the shared-memory image of the MMA B operand
-  const uint8_t* wg_img;  // W_g likewise: the gate is recomputed from LayerNorm(z)
+  // W_o / 2 and W_g / 2 (exact: a power-of-two scale) as shared-memory images of
+  // the MMA B operand; the gate is recomputed from LayerNorm(z)
+  const uint8_t* wo_img;
+  const uint8_t* wg_img;
   const float *b_o, *b_g, *gamma, *beta;
   float eps;
   __nv_bfloat16* out;
@@ -91,6 +93,7 @@ struct GateArgs {
 };
 
 // Device status word values (mirror the public codes).
+constexpr int kStatusBadLaunch = -5;  // TRI_ATTN_ERR_CUDA: a kernel found its launch unusable
 constexpr int kStatusTimeout = -6;
 
 __device__ __forceinline__ void report_status(int* status, int code) {

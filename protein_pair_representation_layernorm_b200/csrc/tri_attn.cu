@@ -700,8 +700,10 @@ int tri_attn_create(const tri_attn_params* p, tri_attn_handle** out) {
   for (float& x : wb) x *= tri::kLog2e;
 
   if (dt == TRI_ATTN_BF16) {
-    // [Wq; Wk; Wv] as 384 K-major rows, Wg and Wo as 128 K-major rows each, all in
-    // the shared-memory image the tcgen05 B operand reads (bf16 bits kept exactly).
+    // [Wq; Wk; Wv] as 384 K-major rows, Wg / 2 and Wo / 2 as 128 K-major rows each,
+    // all in the shared-memory image the tcgen05 B operand reads (bf16 values kept
+    // exactly: halving a bf16 number is exact).  gate_out works with
+    // t = (Wg x + bg) / 2 and a = 2 g o = (1 + tanh t) o, so the halves cancel.
     std::vector<uint16_t> w384(384 * 128), wg128(128 * 128), w128(128 * 128), img;
     const std::vector<float>* parts[3] = {&wq, &wk, &wv};
     for (int part = 0; part < 3; ++part)
@@ -709,9 +711,9 @@ int tri_attn_create(const tri_attn_params* p, tri_attn_handle** out) {
         for (int c = 0; c < kCz; ++c)
           w384[(part * kHD + n) * 128 + c] = f32_to_bf16_bits((*parts[part])[n * kCz + c]);
     for (int n = 0; n < kHD; ++n)
-      for (int c = 0; c < kCz; ++c) wg128[n * 128 + c] = f32_to_bf16_bits(wg[n * kCz + c]);
+      for (int c = 0; c < kCz; ++c) wg128[n * 128 + c] = f32_to_bf16_bits(0.5f * wg[n * kCz + c]);
     for (int n = 0; n < kCz; ++n)
-      for (int c = 0; c < kHD; ++c) w128[n * 128 + c] = f32_to_bf16_bits(wo[n * kHD + c]);
+      for (int c = 0; c < kHD; ++c) w128[n * 128 + c] = f32_to_bf16_bits(0.5f * wo[n * kHD + c]);
     pack_kmajor_sw128(w384, 384, img);
     if ((rc = upload(img, &h->w_qkvg))) return fail(rc);
     pack_kmajor_sw128(wg128, 128, img);
@@ -1059,10 +1061,12 @@ __global__ void pack_weights_noalloc(const bf16* wq, const bf16* wk, const bf16*
       *reinterpret_cast<bf16*>(scratch + kNaWImg + sw128_offset(384, n, k)) = src[nn * kCz + k];
     } else if (idx < n_w + n_wg) {
       const int t = idx - n_w, n = t / 128, k = t % 128;
-      *reinterpret_cast<bf16*>(scratch + kNaWgImg + sw128_offset(128, n, k)) = wg[n * kCz + k];
+      *reinterpret_cast<bf16*>(scratch + kNaWgImg + sw128_offset(128, n, k)) =
+          __float2bfloat16(0.5f * __bfloat162float(wg[n * kCz + k]));  // exact
     } else if (idx < n_w + n_wg + n_wo) {
       const int t = idx - n_w - n_wg, n = t / 128, k = t % 128;
-      *reinterpret_cast<bf16*>(scratch + kNaWoImg + sw128_offset(128, n, k)) = wo[n * kHD + k];
+      *reinterpret_cast<bf16*>(scratch + kNaWoImg + sw128_offset(128, n, k)) =
+          __float2bfloat16(0.5f * __bfloat162float(wo[n * kHD + k]));  // exact
     } else if (idx < n_w + n_wg + n_wo + n_wb) {
       const int t = idx - n_w - n_wg - n_wo;
       reinterpret_cast<float*>(scratch + kNaWb)[t] = __bfloat162float(wb[t]) * tri::kLog2e;
