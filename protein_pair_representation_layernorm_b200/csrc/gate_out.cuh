@@ -33,7 +33,10 @@
 //   4. D_out = A' (Wo/2)^T (8 MMAs) over D_g;
 //   5. out = D_out + bo + z, written over o in the O buffer (128-byte swizzle)
 //      and stored with TMA (through the swapped view again for the ending
-//      node); the O buffer is refilled once the store has read it.
+//      node); the leader refills the O buffer with the group's next tile once
+//      that tile's z has arrived and its copies are issued (by then the store
+//      has read the buffer), which keeps the read-out of the store off the
+//      group's path.
 // Wg/2 and Wo/2 stay resident in shared memory (halving a bf16 weight is
 // exact).  Every element of out is read (as z) and written by the same CTA,
 // tile by tile, so out may alias Z.
@@ -220,6 +223,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 8; ++c)
         tmem_cp_128x256b(t_z + 8 * c, smem_desc(zbuf_u32 + (c >> 2) * kSlabBytes + (c & 3) * 32,
                                                 1024, kSwizzle128B));
+      if (k > 0) {
+        bulk_wait_read_all();  // the previous tile's store has read the O buffer
+        load_o(tile);
+      }
     }
     // ---- x = LayerNorm(z): one pass over this thread's 64 channels (mixed-
     // precision adds widen z exactly), partial sums exchanged with the other
@@ -366,10 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_store_3d(&map_out, obuf + slab * kSlabBytes, 64 * slab, c1, c2);
       bulk_commit();
       stored = true;
-      if (more) {
-        bulk_wait_read_all();  // the O buffer may be refilled after this
-        load_o(tile + tstep);
-      }
+
     }
   }
   if (leader) {
