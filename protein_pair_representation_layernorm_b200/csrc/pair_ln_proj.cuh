@@ -37,6 +37,8 @@
 // This is the HBM-bound step: per pair it reads 256 B and writes 768 B + 8 B.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -337,30 +339,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       // half the two threads of a pair take q and k (4 heads each), after the v
       // half two heads of v each; a chunk is the pair's 64-byte row of that head,
       // written with two 32-byte stores
-      const int nchunks = half == 0 ? kHeads : 2;
       const uint32_t col0 = tmem + lane_base + (half == 0 ? hc * 128 : hc * 64);
       __nv_bfloat16* out = half == 0 ? (hc == 0 ? a.Q : a.K) : a.V;
       const float sc = half == 0 && hc == 0 ? a.q_scale : 1.0f;
-      uint32_t v[32], vn[32];
-      tmem_ld32(col0, vn);
-#pragma unroll 1
-      for (int cc = 0; cc < nchunks; ++cc) {
-        tmem_ld_wait();
+      // every chunk packs into registers of its own, all kept live until the
+      // last store has been issued, so no store waits for the previous one to
+      // release its registers
+      auto chunks = [&](auto nch) {
+        constexpr int kN = decltype(nch)::value;
+        uint32_t pk[kN][16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = vn[e];
-        if (cc + 1 < nchunks) tmem_ld32(col0 + (cc + 1) * 32, vn);  // overlap the next load
-        const int h = half == 0 ? cc : 2 * hc + cc;
-        uint32_t pk[16];
+        for (int cc = 0; cc < kN; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(col0 + cc * 32, v);
+          tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
-        if (jv) {
-          uint32_t* dst = reinterpret_cast<uint32_t*>(
-              out + ((static_cast<long long>(r) * kHeads + h) * a.N + j) * kD);
-          st_global_v8(dst, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
-          st_global_v8(dst + 8, pk[8], pk[9], pk[10], pk[11], pk[12], pk[13], pk[14], pk[15]);
+          for (int e = 0; e < 16; ++e)
+            pk[cc][e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
+          const int h = half == 0 ? cc : 2 * hc + cc;
+          if (jv) {
+            uint32_t* dst = reinterpret_cast<uint32_t*>(
+                out + ((static_cast<long long>(r) * kHeads + h) * a.N + j) * kD);
+            st_global_v8(dst, pk[cc][0], pk[cc][1], pk[cc][2], pk[cc][3], pk[cc][4], pk[cc][5],
+                         pk[cc][6], pk[cc][7]);
+            st_global_v8(dst + 8, pk[cc][8], pk[cc][9], pk[cc][10], pk[cc][11], pk[cc][12],
+                         pk[cc][13], pk[cc][14], pk[cc][15]);
+          }
         }
-      }
+#pragma unroll
+        for (int cc = 0; cc < kN; ++cc)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) asm volatile("" ::"r"(pk[cc][e]));
+      };
+      if (half == 0)
+        chunks(std::integral_constant<int, kHeads>{});
+      else
+        chunks(std::integral_constant<int, 2>{});
       tc_fence_before();
       named_barrier_sync(bar_id, kGroupThreads);  // TMEM (and, after the second half, A) reused
       tc_fence_after();
