@@ -64,6 +64,7 @@ def lib():
         _lib.oracle_pair_features.argtypes = [ctypes.POINTER(_Params), vp, vp, vp, vp, vp]
         _lib.oracle_attend.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, vp, vp]
         _lib.oracle_attend_blockwise.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, vp]
+        _lib.oracle_attend_bwd.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, vp, vp, vp, vp]
         _lib.oracle_tri_attn.argtypes = [ctypes.POINTER(_Params), ci, vp, ci, vp, vp, vp]
         _lib.oracle_num_threads.restype = ci
     return _lib
@@ -194,6 +195,38 @@ def attend_blockwise(q, k, v, bias, mask=None, block=7):
                                        H, d, block, _ptr(o))
     assert rc == 0
     return o
+
+
+def attend_bwd(q, k, v, bias, dout, mask=None):
+    """Gradients (dq, dk, dv, dbias) of attend(q, k, v, bias, mask) given the
+    gradient dout of a loss with respect to its output (shapes as attend)."""
+    q, k, v, bias, dout = _f64(q), _f64(k), _f64(v), _f64(bias), _f64(dout)
+    Nq, H, d = q.shape
+    Nk = k.shape[0]
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    dbias = np.empty((H, Nq, Nk))
+    m = None if mask is None else np.ascontiguousarray(mask, dtype=np.uint8)
+    rc = lib().oracle_attend_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(m), _ptr(dout), Nq,
+                                 Nk, H, d, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbias))
+    assert rc == 0
+    return dq, dk, dv, dbias
+
+
+def tri_attn_core_bwd(q, k, v, bias, dout, mask=None):
+    """Backward of the starting-node attention core over R problem rows, each
+    row an attend() call with its own q, k, v and the shared bias:
+    q, k, v, dout: (R, N, H, d); bias: (H, N, N).  Returns dq, dk, dv
+    (R, N, H, d) and dbias (H, N, N), the bias gradient summed over the rows.
+    (The ending-node core is the same computation on the transposed problem.)"""
+    R = q.shape[0]
+    outs = [attend_bwd(q[r], k[r], v[r], bias, dout[r], mask) for r in range(R)]
+    dq = np.stack([o[0] for o in outs])
+    dk = np.stack([o[1] for o in outs])
+    dv = np.stack([o[2] for o in outs])
+    dbias = np.zeros_like(_f64(bias))
+    for o in outs:
+        dbias += o[3]
+    return dq, dk, dv, dbias
 
 
 def tri_attn(p: Problem, orientation: int, lines=None, bias=None, want_o: bool = False):

@@ -38,6 +38,10 @@
  *  - The mask is a per-residue key mask: a masked residue k contributes
  *    probability exactly 0 as a key; its own rows and columns are still
  *    computed.  If every key is masked, o = 0 and out = z.
+ *  - Training needs the gradients of the attention core with respect to q,
+ *    k, v and the logit bias (BioNeMo context-parallelism page, the training
+ *    setting its context gaps refer to); oracle_attend_bwd writes them out by
+ *    the chain rule through each materialised softmax row.
  *  - Scores are computed on the fly per row; an N x N x H score tensor is
  *    never stored (Design-CP technical summary, §Metodología 1, 2D grid
  *    sharding with ring attention: scores computed without materialising the
@@ -283,6 +287,89 @@ int oracle_attend_blockwise(const double *q, const double *k, const double *v,
       free(acc);
       free(sb);
     }
+  return 0;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Gradients of the attention core (the backward pass).                    */
+
+/* Gradients of oracle_attend with respect to q, k, v and the bias, given the
+ * gradient `dout` of a scalar loss with respect to its output o.  Same shapes
+ * as oracle_attend: q, dq: [Nq][H][d]; k, v, dk, dv: [Nk][H][d]; bias, dbias:
+ * [H][Nq][Nk]; dout: [Nq][H][d].  Every output array is overwritten.
+ *
+ * Plain chain rule through one softmax row (s_k the scaled dot product plus
+ * bias, p = softmax over the unmasked keys, o = sum_k p_k v_k):
+ *   dv_k  += p_k dout                       (o is linear in v)
+ *   dp_k   = dout . v_k                     (d loss / d p_k)
+ *   ds_k   = p_k (dp_k - sum_m p_m dp_m)    (Jacobian of the softmax,
+ *                                            diag(p) - p p^T, applied to dp)
+ *   dbias_k = ds_k,  dq += ds_k k_k / sqrt(d),  dk_k += ds_k q / sqrt(d)
+ * Masked keys have p_k = 0, hence ds_k = 0 and no contribution anywhere; a
+ * query whose every key is masked has o = 0 independent of its inputs and
+ * gets all-zero gradients. */
+int oracle_attend_bwd(const double *q, const double *k, const double *v,
+                      const double *bias, const unsigned char *mask,
+                      const double *dout, int Nq, int Nk, int H, int d,
+                      double *dq, double *dk, double *dv, double *dbias) {
+  if (!q || !k || !v || !bias || !dout || !dq || !dk || !dv || !dbias || Nq < 0 || Nk < 0)
+    return -1;
+  const double scale = 1.0 / sqrt((double)d);
+  memset(dq, 0, sizeof(double) * (size_t)Nq * H * d);
+  memset(dk, 0, sizeof(double) * (size_t)Nk * H * d);
+  memset(dv, 0, sizeof(double) * (size_t)Nk * H * d);
+  memset(dbias, 0, sizeof(double) * (size_t)H * Nq * Nk);
+  double *p = malloc(sizeof(double) * (Nk > 0 ? Nk : 1));
+  double *dp = malloc(sizeof(double) * (Nk > 0 ? Nk : 1));
+  /* sequential: dk and dv collect contributions from every query */
+  for (int h = 0; h < H; ++h)
+    for (int j = 0; j < Nq; ++j) {
+      const double *qj = q + ((long)j * H + h) * d;
+      const double *gj = dout + ((long)j * H + h) * d;
+      double mx = -INFINITY;
+      int any = 0;
+      for (int kk = 0; kk < Nk; ++kk) {
+        if (mask && !mask[kk]) continue;
+        const double *kv = k + ((long)kk * H + h) * d;
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c) dot += qj[c] * kv[c];
+        p[kk] = dot * scale + bias[((long)h * Nq + j) * Nk + kk];
+        if (!any || p[kk] > mx) mx = p[kk];
+        any = 1;
+      }
+      if (!any) continue;
+      double denom = 0.0;
+      for (int kk = 0; kk < Nk; ++kk) {
+        if (mask && !mask[kk]) { p[kk] = 0.0; continue; }
+        p[kk] = exp(p[kk] - mx);
+        denom += p[kk];
+      }
+      double pdp = 0.0; /* sum_m p_m dp_m */
+      for (int kk = 0; kk < Nk; ++kk) {
+        p[kk] /= denom;
+        const double *vv = v + ((long)kk * H + h) * d;
+        double t = 0.0;
+        for (int c = 0; c < d; ++c) t += gj[c] * vv[c];
+        dp[kk] = t;
+        pdp += p[kk] * t;
+      }
+      double *dqj = dq + ((long)j * H + h) * d;
+      for (int kk = 0; kk < Nk; ++kk) {
+        if (p[kk] == 0.0) continue;
+        const double ds = p[kk] * (dp[kk] - pdp);
+        dbias[((long)h * Nq + j) * Nk + kk] = ds;
+        const double *kv = k + ((long)kk * H + h) * d;
+        double *dkk = dk + ((long)kk * H + h) * d;
+        double *dvk = dv + ((long)kk * H + h) * d;
+        for (int c = 0; c < d; ++c) {
+          dqj[c] += ds * kv[c] * scale;
+          dkk[c] += ds * qj[c] * scale;
+          dvk[c] += p[kk] * gj[c];
+        }
+      }
+    }
+  free(p);
+  free(dp);
   return 0;
 }
 
