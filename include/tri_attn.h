@@ -236,6 +236,44 @@ int tri_attn_forward_noalloc(const tri_attn_params *params, const void *Z, int N
                              const uint8_t *mask, tri_attn_orientation orientation, void *out,
                              void *stream, unsigned flags);
 
+/* ---- backward pass of the attention core (fp32) ---------------------------
+ *
+ * Gradients of the starting-node attention core for training (the training
+ * setting of the BioNeMo context-parallelism page).  For R problem rows r,
+ * head h, query j and key k:
+ *   s_jk = q_j . k_k / sqrt(d) + bias[h][j][k]  over keys with mask[k] != 0,
+ *   p = softmax over k,  o_j = sum_k p_jk v_k.
+ * Given dO = d loss / d o, this writes
+ *   dQ_j = sum_k ds_jk k_k / sqrt(d),  dK_k = sum_j ds_jk q_j / sqrt(d),
+ *   dV_k = sum_j p_jk dO_j,  dbias[h][j][k] = sum_r ds_jk,
+ * with ds_jk = p_jk (dO_j . v_k - dO_j . o_j) (the softmax Jacobian applied to
+ * d loss / d p).  Masked keys, and queries whose every key is masked, get zero
+ * gradients.  The ending-node core is this computation on the transposed
+ * problem (its rows are the columns of Z).  Note the natural-unit logits:
+ * q is not pre-scaled and the bias is not multiplied by log2(e), unlike the
+ * forward's workspace.
+ *
+ * Layouts (device memory, fp32, contiguous): Q, K, V, dO, dQ, dK, dV
+ * [rows][H][N][d] with H = 4, d = 32 (the head-major layout of the forward's
+ * workspace); bias, dbias [H][N][N]; mask [N] (1 = valid key) or NULL.
+ * Q, K, V, dO, dQ, dK, dV and workspace must be 16-byte aligned.  The caller
+ * owns every buffer; the call allocates nothing.  `workspace` holds the row
+ * statistics and must have at least
+ * tri_attn_attention_backward_workspace_bytes(rows, N) bytes.
+ * Asynchronous on `stream` (four kernel launches, SIMT fp32 arithmetic: each
+ * gradient agrees with an fp64 evaluation to ~1e-6 relative); dbias is written
+ * once per element (no atomics), so the result is deterministic.
+ * Errors: TRI_ATTN_ERR_INVALID_ARG (NULL or misaligned pointer, rows or N < 1,
+ * workspace too small), TRI_ATTN_ERR_UNSUPPORTED (rows > 65535 or N > 46340),
+ * TRI_ATTN_ERR_NO_DEVICE, TRI_ATTN_ERR_CUDA (launch failure).
+ * Flags: TRI_ATTN_FLAG_SYNC synchronises the stream before returning. */
+size_t tri_attn_attention_backward_workspace_bytes(int rows, int N);
+int tri_attn_attention_backward(const float *Q, const float *K, const float *V,
+                                const float *bias, const uint8_t *mask, const float *dO,
+                                int rows, int N, float *dQ, float *dK, float *dV,
+                                float *dbias, void *workspace, size_t workspace_bytes,
+                                void *stream, unsigned flags);
+
 /* Release everything the handle owns.  NULL-safe.  Not stream-ordered:
  * call it after the work that uses the handle has completed. */
 int tri_attn_destroy(tri_attn_handle *h);

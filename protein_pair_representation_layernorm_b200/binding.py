@@ -94,6 +94,10 @@ def lib() -> ctypes.CDLL:
         L.tri_attn_bias_ld.argtypes = [ci]
         L.tri_attn_rows_bias.argtypes = [vp, vp, ci, ci, ci, vp, vp, vp, cu]
         L.tri_attn_rows_forward.argtypes = [vp, vp, ci, ci, ci, vp, vp, vp, vp, cu]
+        L.tri_attn_attention_backward_workspace_bytes.argtypes = [ci, ci]
+        L.tri_attn_attention_backward_workspace_bytes.restype = sz
+        L.tri_attn_attention_backward.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, vp, vp, vp, vp,
+                                                  vp, sz, vp, cu]
         L.tri_attn_destroy.argtypes = [vp]
         L.tri_attn_status_string.argtypes = [ci]
         L.tri_attn_status_string.restype = ctypes.c_char_p
@@ -178,6 +182,18 @@ def tri_attn_forward_noalloc(params: tri_attn_params, Z_ptr, N: int, mask_ptr, o
 
 def tri_attn_destroy(h) -> int:
     return lib().tri_attn_destroy(h)
+
+
+def tri_attn_attention_backward_workspace_bytes(rows: int, N: int) -> int:
+    return int(lib().tri_attn_attention_backward_workspace_bytes(int(rows), int(N)))
+
+
+def tri_attn_attention_backward(Q, K, V, bias, mask, dO, rows: int, N: int, dQ, dK, dV, dbias,
+                                workspace, workspace_bytes: int, stream=None, flags: int = 0) -> int:
+    """Backward pass of the attention core (device pointers); see tri_attn.h."""
+    return lib().tri_attn_attention_backward(Q, K, V, bias, mask, dO, int(rows), int(N), dQ, dK,
+                                             dV, dbias, workspace, int(workspace_bytes), stream,
+                                             int(flags))
 
 
 # ---------------------------------------------------------------- convenience
@@ -311,3 +327,31 @@ class TriangleAttention:
             self.close()
         except Exception:
             pass
+
+
+def attention_backward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, bias: torch.Tensor,
+                       dO: torch.Tensor, mask: torch.Tensor | None = None, stream=None):
+    """Gradients (dQ, dK, dV, dbias) of the attention core on the GPU.
+
+    Q, K, V, dO: fp32 CUDA tensors [rows][H][N][d] (H = 4, d = 32); bias: fp32
+    [H][N][N] (natural-unit logits); mask: uint8 [N] or None.  Allocates the
+    outputs and the row-statistics workspace with torch and calls
+    tri_attn_attention_backward on `stream` (default: the current stream)."""
+    rows, H, N, d = Q.shape
+    for t in (Q, K, V, dO):
+        if t.dtype != torch.float32 or not t.is_cuda or tuple(t.shape) != (rows, H, N, d):
+            raise ValueError("Q, K, V, dO must be fp32 CUDA tensors of one shape [rows][H][N][d]")
+    if bias.dtype != torch.float32 or tuple(bias.shape) != (H, N, N):
+        raise ValueError("bias must be an fp32 CUDA tensor [H][N][N]")
+    Q, K, V, dO, bias = (t.contiguous() for t in (Q, K, V, dO, bias))
+    m = None if mask is None else mask.to(device=Q.device, dtype=torch.uint8).contiguous()
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    dB = torch.empty_like(bias)
+    nbytes = tri_attn_attention_backward_workspace_bytes(rows, N)
+    ws = torch.empty(max(nbytes // 4, 4), dtype=torch.float32, device=Q.device)
+    rc = tri_attn_attention_backward(_ptr(Q), _ptr(K), _ptr(V), _ptr(bias), _ptr(m), _ptr(dO),
+                                     rows, N, _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dB), _ptr(ws),
+                                     ws.numel() * 4, _stream_handle(stream), 0)
+    if rc != TRI_ATTN_OK:
+        raise TriAttnError(rc, "tri_attn_attention_backward")
+    return dQ, dK, dV, dB

@@ -5,7 +5,8 @@
 //   pair_ln_proj  (LayerNorm + Q/K/V/gate/bias, tcgen05)        HBM-bound
 //   tri_attn_fwd  (online-softmax attention, tcgen05 + TMA)     tensor/ALU-bound
 //   gate_out      (gate * o, output projection, residual)       HBM-bound
-// (fp32 handles run the SIMT kernels of kernels_f32.cuh instead).  The logit
+// (fp32 handles run the SIMT kernels of kernels_f32.cuh instead; the backward
+// pass of the attention core runs the kernels of attn_bwd.cuh).  The logit
 // bias of every pair is needed by every row, so it is produced for all pairs
 // before any attention runs; when the workspace for all rows exceeds the
 // handle's limit, a bias-only pass runs first and the rest proceeds in row
@@ -25,6 +26,7 @@
 #include <new>
 #include <vector>
 
+#include "attn_bwd.cuh"
 #include "common.cuh"
 #include "gate_out.cuh"
 #include "kernels_f32.cuh"
@@ -1172,4 +1174,60 @@ extern "C" int tri_attn_forward_noalloc(const tri_attn_params* p, const void* Z,
   }
   hh.ws = nullptr;  // nothing in hh is owned: the handle is never destroyed
   return rc;
+}
+
+// ------------------------------------------------------------------ backward
+// The backward pass of the attention core (attn_bwd.cuh): row statistics, then
+// dQ, dK/dV and the bias gradient, four launches on the caller's stream.
+
+extern "C" size_t tri_attn_attention_backward_workspace_bytes(int rows, int N) {
+  if (rows < 1 || N < 1) return 0;
+  return 2 * static_cast<size_t>(rows) * tri::kHeads * N * sizeof(float);
+}
+
+extern "C" int tri_attn_attention_backward(const float* Q, const float* K, const float* V,
+                                           const float* bias, const uint8_t* mask,
+                                           const float* dO, int rows, int N, float* dQ,
+                                           float* dK, float* dV, float* dbias, void* workspace,
+                                           size_t workspace_bytes, void* stream,
+                                           unsigned flags) {
+  const void* vec[] = {Q, K, V, dO, dQ, dK, dV, workspace};
+  for (const void* ptr : vec)
+    if (!ptr || reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return TRI_ATTN_ERR_INVALID_ARG;
+  if (!bias || !dbias || rows < 1 || N < 1) return TRI_ATTN_ERR_INVALID_ARG;
+  // indices stay within 64-bit element offsets; grids within their limits
+  if (rows > 65535 || N > 46340) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (workspace_bytes < tri_attn_attention_backward_workspace_bytes(rows, N))
+    return TRI_ATTN_ERR_INVALID_ARG;
+  int rc = check_device();
+  if (rc != TRI_ATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  tri::bwd::BwdArgs a{};
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.B = bias;
+  a.dO = dO;
+  a.mask = mask;
+  a.dQ = dQ;
+  a.dK = dK;
+  a.dV = dV;
+  a.dB = dbias;
+  a.lse = static_cast<float*>(workspace);
+  a.D = a.lse + static_cast<size_t>(rows) * tri::kHeads * N;
+  a.rows = rows;
+  a.N = N;
+  const unsigned tiles = static_cast<unsigned>((N + tri::bwd::kThreadsRow - 1) / tri::bwd::kThreadsRow);
+  const dim3 grid_rows(tiles, static_cast<unsigned>(rows), tri::kHeads);
+  tri::bwd::bwd_stats<<<grid_rows, tri::bwd::kThreadsRow, 0, st>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  tri::bwd::bwd_dq<<<grid_rows, tri::bwd::kThreadsRow, 0, st>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  tri::bwd::bwd_dkdv<<<grid_rows, tri::bwd::kThreadsRow, 0, st>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  const unsigned blocks = static_cast<unsigned>((N + tri::bwd::kBlk - 1) / tri::bwd::kBlk);
+  tri::bwd::bwd_dbias<<<dim3(blocks, blocks, tri::kHeads), tri::bwd::kBlkThreads, 0, st>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  if (flags & TRI_ATTN_FLAG_SYNC) CUDA_TRY(cudaStreamSynchronize(st));
+  return TRI_ATTN_OK;
 }

@@ -117,3 +117,28 @@ def test_binding_constants_match_the_header():
     assert len(defs) >= 14
     for name, value in defs:
         assert getattr(binding, name) == int(value), name
+
+
+def test_attention_backward_rejects_bad_arguments_without_device():
+    L = binding.lib()
+    ws_bytes = binding.tri_attn_attention_backward_workspace_bytes
+    assert ws_bytes(0, 10) == 0 and ws_bytes(3, 0) == 0
+    assert ws_bytes(3, 70) == 2 * 3 * 4 * 70 * 4  # log-sum-exp and D per (row, head, query)
+    buf = 0x10000
+    ok = dict(Q=buf, K=buf, V=buf, bias=buf, mask=None, dO=buf, rows=3, N=70, dQ=buf, dK=buf,
+              dV=buf, dbias=buf, workspace=buf, workspace_bytes=ws_bytes(3, 70), stream=None,
+              flags=0)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return L.tri_attn_attention_backward(*a.values())
+
+    assert call(Q=None) == binding.TRI_ATTN_ERR_INVALID_ARG
+    assert call(dbias=None) == binding.TRI_ATTN_ERR_INVALID_ARG
+    assert call(dK=buf + 4) == binding.TRI_ATTN_ERR_INVALID_ARG  # misaligned
+    assert call(rows=0) == binding.TRI_ATTN_ERR_INVALID_ARG
+    assert call(N=0) == binding.TRI_ATTN_ERR_INVALID_ARG
+    assert call(workspace_bytes=ws_bytes(3, 70) - 4) == binding.TRI_ATTN_ERR_INVALID_ARG
+    assert call(N=46341, workspace_bytes=ws_bytes(3, 46341)) == binding.TRI_ATTN_ERR_UNSUPPORTED
+    if not torch.cuda.is_available():
+        assert call() == binding.TRI_ATTN_ERR_NO_DEVICE
