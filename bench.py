@@ -69,6 +69,8 @@ def parse():
     ap.add_argument("--workload", type=int, default=WORKLOAD,
                     help="workload index (the metric is quoted on the default; others are for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the attention-core backward (fp32) instead; one JSON line")
     return ap.parse_args()
 
 
@@ -395,11 +397,70 @@ def run_ours(args, world, rank, local):
     blk.close()
 
 
+def run_backward(args, rank):
+    """Time tri_attn_attention_backward (fp32 SIMT kernels) on the workload's N
+    with every row, on synthetic q, k, v, dO and bias; prints one JSON line.
+    Algorithmic work: 10 d flop per (row, head, query, unmasked key) score
+    (S and dP, 2 d each, recomputed once; dQ, dK and dV, 2 d each)."""
+    if rank != 0:
+        return
+    import ctypes
+
+    from protein_pair_representation_layernorm_b200 import binding, workloads
+    w = workloads.WORKLOADS[args.workload]
+    inp = workloads.workload_inputs(args.workload)
+    N = inp.N
+    rows = N
+    H, d = 4, 32
+    gen = torch.Generator(device="cuda").manual_seed(17)
+    Q, K, V, dO = (torch.randn(rows, H, N, d, device="cuda", generator=gen) for _ in range(4))
+    bias = torch.randn(H, N, N, device="cuda", generator=gen)
+    mask = None if inp.mask is None else inp.mask.cuda().to(torch.uint8).contiguous()
+    n_valid = N if inp.mask is None else int(inp.mask.sum())
+    dQ, dK, dV, dB = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(bias)
+    nbytes = binding.tri_attn_attention_backward_workspace_bytes(rows, N)
+    ws = torch.empty(nbytes // 4, dtype=torch.float32, device="cuda")
+    st = torch.cuda.Stream()
+    P = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())  # noqa: E731
+
+    def step():
+        rc = binding.tri_attn_attention_backward(P(Q), P(K), P(V), P(bias), P(mask), P(dO), rows, N,
+                                                 P(dQ), P(dK), P(dV), P(dB), P(ws), nbytes,
+                                                 ctypes.c_void_p(st.cuda_stream), 0)
+        assert rc == binding.TRI_ATTN_OK, binding.tri_attn_status_string(rc)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    st.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(st)
+    for _ in range(args.steps):
+        step()
+    ev1.record(st)
+    ev1.synchronize()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    flops = 10.0 * d * rows * N * n_valid * H
+    tf = flops / (ms / 1e3) / 1e12
+    # fp32 FFMA peak: 148 SMs x 128 lanes x 2 flop x 1965 MHz
+    peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    print(json.dumps({
+        "metric": "attention-core backward TFLOP/s (algorithmic: 10 d flop per unmasked score)",
+        "value": tf, "unit": "TFLOP/s", "ms_per_step": ms, "steps": args.steps,
+        "warmup": max(args.warmup, 1), "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "N": N, "rows": rows, "heads": H, "head_dim": d},
+        "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tf / peak,
+                     "peak_derivation": "fp32 FFMA: 148 SMs x 128 lanes x 2 flop x 1965 MHz"},
+        "gpu_launches": 4 * args.steps}), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
     try:
-        if args.impl == "reference":
+        if args.backward:
+            run_backward(args, rank)
+        elif args.impl == "reference":
             run_reference(args, world, rank)
         else:
             run_ours(args, world, rank, local)
