@@ -136,6 +136,32 @@ int tri_attn_forward_host(tri_attn_handle *h, const void *Z_host, int N,
                           int n_orientations, void *out_host, void *stream,
                           unsigned flags);
 
+/* Asynchronous form of tri_attn_forward_host, for a stream of independent
+ * problems: same arguments and result, but the call returns once the copies
+ * and the blocks are enqueued.  The uploads run on a copy stream of the
+ * handle, the blocks on `stream`, the downloads on a second copy stream of the
+ * handle, ordered by events; the handle keeps three device staging buffers
+ * (allocated on first use, each N x N x c_z elements), so consecutive calls
+ * overlap one call's upload, another's computation and a third's download
+ * (PCIe carries both directions at once).
+ * Rules: every asynchronous call on a handle uses the same `stream`; Z_host,
+ * mask_host and out_host must stay valid and unmodified until
+ * tri_attn_host_wait returns; one in-flight call's out_host must not be
+ * another in-flight call's Z_host (a call's own Z_host may be its out_host;
+ * in-flight calls may share one out_host: the downloads run in call order).
+ * A call with a larger N than before waits for the calls in flight first.
+ * Errors are those of tri_attn_forward_host, returned by the call that
+ * detects them; device errors (a timed-out wait) by tri_attn_host_wait. */
+int tri_attn_forward_host_async(tri_attn_handle *h, const void *Z_host, int N,
+                                const uint8_t *mask_host, const int *orientations,
+                                int n_orientations, void *out_host, void *stream,
+                                unsigned flags);
+
+/* Wait until every tri_attn_forward_host_async call on the handle has
+ * completed (its results are in out_host) and return the sticky device status
+ * (TRI_ATTN_OK or TRI_ATTN_ERR_TIMEOUT), then clear it. */
+int tri_attn_host_wait(tri_attn_handle *h);
+
 /* Synchronise `stream` and return the sticky device status of the handle
  * (TRI_ATTN_OK or TRI_ATTN_ERR_TIMEOUT), then clear it. */
 int tri_attn_get_status(tri_attn_handle *h, void *stream);

@@ -81,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.tri_attn_create.argtypes = [ctypes.POINTER(tri_attn_params), ctypes.POINTER(vp)]
         L.tri_attn_forward.argtypes = [vp, vp, ci, vp, ci, vp, vp, cu]
         L.tri_attn_forward_host.argtypes = [vp, vp, ci, vp, vp, ci, vp, vp, cu]
+        L.tri_attn_forward_host_async.argtypes = [vp, vp, ci, vp, vp, ci, vp, vp, cu]
+        L.tri_attn_host_wait.argtypes = [vp]
         L.tri_attn_get_status.argtypes = [vp, vp]
         L.tri_attn_kernel_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float),
                                             ctypes.POINTER(ctypes.c_int)]
@@ -140,6 +142,17 @@ def tri_attn_forward_host(h, Z_host_ptr: int, N: int, mask_host_ptr, orientation
     arr = (ctypes.c_int * len(orientations))(*[int(o) for o in orientations])
     return lib().tri_attn_forward_host(h, Z_host_ptr, int(N), mask_host_ptr, arr,
                                        len(orientations), out_host_ptr, stream, int(flags))
+
+
+def tri_attn_forward_host_async(h, Z_host_ptr: int, N: int, mask_host_ptr, orientations,
+                                out_host_ptr: int, stream: int = 0, flags: int = 0) -> int:
+    arr = (ctypes.c_int * len(orientations))(*[int(o) for o in orientations])
+    return lib().tri_attn_forward_host_async(h, Z_host_ptr, int(N), mask_host_ptr, arr,
+                                             len(orientations), out_host_ptr, stream, int(flags))
+
+
+def tri_attn_host_wait(h) -> int:
+    return lib().tri_attn_host_wait(h)
 
 
 def tri_attn_get_status(h, stream: int = 0) -> int:
@@ -262,6 +275,30 @@ class TriangleAttention:
         if rc != TRI_ATTN_OK:
             raise TriAttnError(rc, "tri_attn_forward_host")
         return out
+
+    def forward_host_async(self, Z_host: torch.Tensor, orientations, mask=None,
+                           out: torch.Tensor | None = None, stream=None, flags: int = 0):
+        """Enqueue tri_attn_forward_host_async; the result is in `out` after
+        host_wait().  The tensors must stay alive and unmodified until then."""
+        assert not Z_host.is_cuda and Z_host.is_contiguous()
+        if out is None:
+            out = torch.empty_like(Z_host)
+        if mask is not None:
+            mask = mask.to(torch.uint8).contiguous()
+        keep = getattr(self, "_async_keep", [])
+        keep.append((Z_host, out, mask))  # alive until host_wait
+        self._async_keep = keep
+        rc = tri_attn_forward_host_async(self.handle, _ptr(Z_host), Z_host.shape[0], _ptr(mask),
+                                         list(orientations), _ptr(out), _stream_handle(stream),
+                                         flags)
+        if rc != TRI_ATTN_OK:
+            raise TriAttnError(rc, "tri_attn_forward_host_async")
+        return out
+
+    def host_wait(self) -> int:
+        rc = tri_attn_host_wait(self.handle)
+        self._async_keep = []
+        return rc
 
     # ---- row-sharded execution (bf16): see tri_attn_rows_bias / _forward in
     # include/tri_attn.h.  Z_rows is the slab of problem rows row0.. of an

@@ -220,16 +220,23 @@ struct tri_attn_handle {
   // last forward, for tri_attn_debug_workspace
   void *q = nullptr, *k = nullptr, *v = nullptr, *g = nullptr, *bias = nullptr, *o = nullptr;
   int ld_bias = 0, rows_last = 0;
-  // host-buffer entry point staging
-  void* stage = nullptr;
-  size_t stage_bytes = 0;
+  // host-buffer entry points: a ring of device staging buffers (allocated on
+  // first use), so that consecutive asynchronous calls overlap one call's
+  // upload, another's computation and a third's download
+  static constexpr int kRing = 3;
+  void* stage[kRing] = {};
+  size_t stage_bytes = 0;      // size of each staging buffer
+  long long ring_next = 0;     // asynchronous calls issued
+  cudaEvent_t slot_free[kRing] = {};  // recorded after the last download from the slot
+  bool slot_pending[kRing] = {};
   uint8_t* stage_mask = nullptr;
   size_t stage_mask_bytes = 0;
-  // forward_host: the stream its read-back copies run on, and the event that
-  // orders each copy after the chunk that produced it
-  cudaStream_t copy_st = nullptr;
-  cudaEvent_t chunk_ev = nullptr;
-  static constexpr int kInRanges = 8;  // input copies of forward_host, one event each
+  // the streams the uploads and the downloads run on, and the events that order
+  // the computation after each uploaded piece and each download after the chunk
+  // that produced it
+  cudaStream_t copy_in = nullptr, copy_out = nullptr;
+  cudaEvent_t chunk_ev = nullptr, up_ev = nullptr;
+  static constexpr int kInRanges = 8;  // pieces of the upload, one event each
   cudaEvent_t in_ev[kInRanges] = {};
   // kernel timing
   std::vector<EventPair> ev[3];
@@ -825,29 +832,57 @@ int tri_attn_rows_forward(tri_attn_handle* h, const void* Z_rows, int N, int row
   return finish_call(h, st, flags);
 }
 
-int tri_attn_forward_host(tri_attn_handle* h, const void* Z_host, int N, const uint8_t* mask_host,
-                          const int* orientations, int n_orientations, void* out_host,
-                          void* stream, unsigned flags) {
-  if (!h || !Z_host || !out_host || N < 1 || n_orientations < 0 ||
-      (n_orientations > 0 && !orientations))
-    return TRI_ATTN_ERR_INVALID_ARG;
-  for (int t = 0; t < n_orientations; ++t)
-    if (orientations[t] != TRI_ATTN_STARTING && orientations[t] != TRI_ATTN_ENDING)
-      return TRI_ATTN_ERR_INVALID_ARG;
-  if (N > 46340) return TRI_ATTN_ERR_UNSUPPORTED;
-  if (cudaSetDevice(h->device) != cudaSuccess) return TRI_ATTN_ERR_CUDA;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+}  // extern "C"
+
+namespace {
+
+// Wait for every upload and download of the host-buffer entry points.
+int host_drain(tri_attn_handle* h) {
+  const cudaError_t a = h->copy_in ? cudaStreamSynchronize(h->copy_in) : cudaSuccess;
+  const cudaError_t b = h->copy_out ? cudaStreamSynchronize(h->copy_out) : cudaSuccess;
+  for (bool& p : h->slot_pending) p = false;
+  return a == cudaSuccess && b == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
+}
+
+// The host-buffer forward, enqueued on three streams: uploads on copy_in, the
+// blocks on `st`, downloads on copy_out, ordered by events.  `slot` picks the
+// device staging buffer; the upload into it waits for the slot's previous
+// download.  Returns once everything is enqueued.
+int host_enqueue(tri_attn_handle* h, const void* Z_host, int N, const uint8_t* mask_host,
+                 const int* orientations, int n_orientations, void* out_host, cudaStream_t st,
+                 unsigned flags, int slot) {
   const size_t bytes = static_cast<size_t>(N) * N * kCz * esize(h->dtype);
+  if (!h->copy_in) CUDA_TRY(cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking));
+  if (!h->copy_out) CUDA_TRY(cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking));
+  if (!h->chunk_ev) CUDA_TRY(cudaEventCreateWithFlags(&h->chunk_ev, cudaEventDisableTiming));
+  if (!h->up_ev) CUDA_TRY(cudaEventCreateWithFlags(&h->up_ev, cudaEventDisableTiming));
+  for (int k = 0; k < tri_attn_handle::kRing; ++k)
+    if (!h->slot_free[k])
+      CUDA_TRY(cudaEventCreateWithFlags(&h->slot_free[k], cudaEventDisableTiming));
   if (h->stage_bytes < bytes) {
-    if (h->stage) cudaFree(h->stage);
-    h->stage = nullptr;
-    h->stage_bytes = 0;
-    CUDA_TRY(cudaMalloc(&h->stage, bytes));
+    // a larger problem: every staging buffer is reallocated once nothing uses it
+    const int rc = host_drain(h);
+    if (rc != TRI_ATTN_OK) return rc;
+    CUDA_TRY(cudaStreamSynchronize(st));
+    for (void*& b : h->stage) {
+      if (b) cudaFree(b);
+      b = nullptr;
+    }
     h->stage_bytes = bytes;
   }
+  if (!h->stage[slot]) {
+    const cudaError_t e = cudaMalloc(&h->stage[slot], h->stage_bytes);
+    if (e != cudaSuccess) {
+      h->stage[slot] = nullptr;
+      return e == cudaErrorMemoryAllocation ? TRI_ATTN_ERR_OOM : TRI_ATTN_ERR_CUDA;
+    }
+  }
+  char* stage = static_cast<char*>(h->stage[slot]);
   const uint8_t* dmask = nullptr;
   if (mask_host) {
+    // on `st`: ordered after the previous call's blocks, which read the buffer
     if (h->stage_mask_bytes < static_cast<size_t>(N)) {
+      CUDA_TRY(cudaStreamSynchronize(st));
       if (h->stage_mask) cudaFree(h->stage_mask);
       h->stage_mask = nullptr;
       h->stage_mask_bytes = 0;
@@ -857,15 +892,14 @@ int tri_attn_forward_host(tri_attn_handle* h, const void* Z_host, int N, const u
     CUDA_TRY(cudaMemcpyAsync(h->stage_mask, mask_host, N, cudaMemcpyHostToDevice, st));
     dmask = h->stage_mask;
   }
-  if (!h->copy_st) CUDA_TRY(cudaStreamCreateWithFlags(&h->copy_st, cudaStreamNonBlocking));
-  if (!h->chunk_ev) CUDA_TRY(cudaEventCreateWithFlags(&h->chunk_ev, cudaEventDisableTiming));
+  // the slot's previous download must be complete before the upload overwrites it
+  if (h->slot_pending[slot]) CUDA_TRY(cudaStreamWaitEvent(h->copy_in, h->slot_free[slot], 0));
   const size_t es = esize(h->dtype), pair_b = kCz * es, row_b = static_cast<size_t>(N) * pair_b;
-  // With two or more blocks and an unchunked bf16 first block, Z goes to the
-  // device in kInRanges pieces on the copy stream (rows of Z when the first
-  // block is a starting node, columns when it is an ending node), and the
-  // first block's projection of each piece starts as soon as that piece has
-  // arrived; everything after the projection needs the whole bias and waits
-  // for all pieces.
+  // With two or more blocks and an unchunked bf16 first block, Z goes up in
+  // kInRanges pieces (rows of Z when the first block is a starting node,
+  // columns when it is an ending node), and the first block's projection of
+  // each piece starts as soon as that piece has arrived; everything after the
+  // projection needs the whole bias and waits for all pieces.
   const bool pipelined_in = n_orientations >= 2 && h->dtype == TRI_ATTN_BF16 &&
                             layout_for(h->dtype, N, N).total <= h->ws_limit &&
                             N >= tri_attn_handle::kInRanges;
@@ -876,25 +910,28 @@ int tri_attn_forward_host(tri_attn_handle* h, const void* Z_host, int N, const u
       if (!h->in_ev[c]) CUDA_TRY(cudaEventCreateWithFlags(&h->in_ev[c], cudaEventDisableTiming));
       const int r0 = c * in_split, nr = std::min(in_split, N - r0);
       if (nr <= 0) continue;
-      char* dst = static_cast<char*>(h->stage);
       const char* src = static_cast<const char*>(Z_host);
       if (first == TRI_ATTN_STARTING) {
-        CUDA_TRY(cudaMemcpyAsync(dst + r0 * row_b, src + r0 * row_b, nr * row_b,
-                                 cudaMemcpyHostToDevice, h->copy_st));
+        CUDA_TRY(cudaMemcpyAsync(stage + r0 * row_b, src + r0 * row_b, nr * row_b,
+                                 cudaMemcpyHostToDevice, h->copy_in));
       } else {  // columns r0 .. r0+nr-1 of every row
-        CUDA_TRY(cudaMemcpy2DAsync(dst + r0 * pair_b, row_b, src + r0 * pair_b, row_b,
+        CUDA_TRY(cudaMemcpy2DAsync(stage + r0 * pair_b, row_b, src + r0 * pair_b, row_b,
                                    nr * pair_b, static_cast<size_t>(N), cudaMemcpyHostToDevice,
-                                   h->copy_st));
+                                   h->copy_in));
       }
-      CUDA_TRY(cudaEventRecord(h->in_ev[c], h->copy_st));
+      CUDA_TRY(cudaEventRecord(h->in_ev[c], h->copy_in));
     }
   } else {
-    CUDA_TRY(cudaMemcpyAsync(h->stage, Z_host, bytes, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(cudaMemcpyAsync(stage, Z_host, bytes, cudaMemcpyHostToDevice, h->copy_in));
+    CUDA_TRY(cudaEventRecord(h->up_ev, h->copy_in));
+    CUDA_TRY(cudaStreamWaitEvent(st, h->up_ev, 0));
   }
   if (n_orientations == 0) {
-    CUDA_TRY(cudaMemcpyAsync(out_host, h->stage, bytes, cudaMemcpyDeviceToHost, st));
-    CUDA_TRY(cudaStreamSynchronize(st));
-    return read_status(h, st);
+    CUDA_TRY(cudaStreamWaitEvent(h->copy_out, h->up_ev, 0));
+    CUDA_TRY(cudaMemcpyAsync(out_host, stage, bytes, cudaMemcpyDeviceToHost, h->copy_out));
+    CUDA_TRY(cudaEventRecord(h->slot_free[slot], h->copy_out));
+    h->slot_pending[slot] = true;
+    return TRI_ATTN_OK;
   }
   for (int t = 0; t + 1 < n_orientations; ++t) {
     ChunkHook in_hook;
@@ -905,44 +942,98 @@ int tri_attn_forward_host(tri_attn_handle* h, const void* Z_host, int N, const u
         return TRI_ATTN_OK;
       };
     }
-    int rc = forward_impl(h, h->stage, N, dmask, orientations[t], h->stage, st,
-                          flags & ~TRI_ATTN_FLAG_SYNC, nullptr,
-                          (t == 0 && pipelined_in) ? &in_hook : nullptr);
-    if (rc != TRI_ATTN_OK) {
-      cudaStreamSynchronize(h->copy_st);
-      return rc;
-    }
+    const int rc = forward_impl(h, stage, N, dmask, orientations[t], stage, st,
+                                flags & ~TRI_ATTN_FLAG_SYNC, nullptr,
+                                (t == 0 && pipelined_in) ? &in_hook : nullptr);
+    if (rc != TRI_ATTN_OK) return rc;
   }
   // The last block runs in row chunks (about 8), and each chunk's output goes
-  // back to the host on a second stream as soon as its gate_out has run, while
-  // the later chunks compute: a chunk's output region (rows of Z for the
-  // starting node, columns for the ending node) is final once written, and no
-  // later chunk reads or writes it.
+  // back to the host on copy_out as soon as its gate_out has run, while the
+  // later chunks compute: a chunk's output region (rows of Z for the starting
+  // node, columns for the ending node) is final once written, and no later
+  // chunk reads or writes it.
   const int last = orientations[n_orientations - 1];
   ChunkHook hook;
   hook.max_rows = std::max(tri::attn::kRows,
                            ((N + 7) / 8 + tri::attn::kRows - 1) / tri::attn::kRows * tri::attn::kRows);
   hook.after = [&](int r0, int nr) -> int {
     CUDA_TRY(cudaEventRecord(h->chunk_ev, st));
-    CUDA_TRY(cudaStreamWaitEvent(h->copy_st, h->chunk_ev, 0));
+    CUDA_TRY(cudaStreamWaitEvent(h->copy_out, h->chunk_ev, 0));
     char* dst = static_cast<char*>(out_host);
-    const char* src = static_cast<const char*>(h->stage);
     if (last == TRI_ATTN_STARTING) {
-      CUDA_TRY(cudaMemcpyAsync(dst + r0 * row_b, src + r0 * row_b, nr * row_b,
-                               cudaMemcpyDeviceToHost, h->copy_st));
+      CUDA_TRY(cudaMemcpyAsync(dst + r0 * row_b, stage + r0 * row_b, nr * row_b,
+                               cudaMemcpyDeviceToHost, h->copy_out));
     } else {  // columns r0 .. r0+nr-1 of every row
-      CUDA_TRY(cudaMemcpy2DAsync(dst + r0 * pair_b, row_b, src + r0 * pair_b, row_b, nr * pair_b,
-                                 static_cast<size_t>(N), cudaMemcpyDeviceToHost, h->copy_st));
+      CUDA_TRY(cudaMemcpy2DAsync(dst + r0 * pair_b, row_b, stage + r0 * pair_b, row_b,
+                                 nr * pair_b, static_cast<size_t>(N), cudaMemcpyDeviceToHost,
+                                 h->copy_out));
     }
     return TRI_ATTN_OK;
   };
-  int rc = forward_impl(h, h->stage, N, dmask, last, h->stage, st, flags & ~TRI_ATTN_FLAG_SYNC,
-                        nullptr, &hook);
-  const cudaError_t e_copy = cudaStreamSynchronize(h->copy_st);
+  const int rc = forward_impl(h, stage, N, dmask, last, stage, st, flags & ~TRI_ATTN_FLAG_SYNC,
+                              nullptr, &hook);
   if (rc != TRI_ATTN_OK) return rc;
-  if (e_copy != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+  CUDA_TRY(cudaEventRecord(h->slot_free[slot], h->copy_out));
+  h->slot_pending[slot] = true;
+  return TRI_ATTN_OK;
+}
+
+int host_check(tri_attn_handle* h, const void* Z_host, int N, const int* orientations,
+               int n_orientations, const void* out_host) {
+  if (!h || !Z_host || !out_host || N < 1 || n_orientations < 0 ||
+      (n_orientations > 0 && !orientations))
+    return TRI_ATTN_ERR_INVALID_ARG;
+  for (int t = 0; t < n_orientations; ++t)
+    if (orientations[t] != TRI_ATTN_STARTING && orientations[t] != TRI_ATTN_ENDING)
+      return TRI_ATTN_ERR_INVALID_ARG;
+  if (N > 46340) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (cudaSetDevice(h->device) != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+  return TRI_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int tri_attn_forward_host(tri_attn_handle* h, const void* Z_host, int N, const uint8_t* mask_host,
+                          const int* orientations, int n_orientations, void* out_host,
+                          void* stream, unsigned flags) {
+  int rc = host_check(h, Z_host, N, orientations, n_orientations, out_host);
+  if (rc != TRI_ATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = host_enqueue(h, Z_host, N, mask_host, orientations, n_orientations, out_host, st, flags,
+                    0);
+  const int rd = host_drain(h);
+  if (rc != TRI_ATTN_OK) {
+    cudaStreamSynchronize(st);
+    return rc;
+  }
+  if (rd != TRI_ATTN_OK) return rd;
   CUDA_TRY(cudaStreamSynchronize(st));
   return read_status(h, st);
+}
+
+int tri_attn_forward_host_async(tri_attn_handle* h, const void* Z_host, int N,
+                                const uint8_t* mask_host, const int* orientations,
+                                int n_orientations, void* out_host, void* stream,
+                                unsigned flags) {
+  int rc = host_check(h, Z_host, N, orientations, n_orientations, out_host);
+  if (rc != TRI_ATTN_OK) return rc;
+  const int slot = static_cast<int>(h->ring_next % tri_attn_handle::kRing);
+  rc = host_enqueue(h, Z_host, N, mask_host, orientations, n_orientations, out_host,
+                    static_cast<cudaStream_t>(stream), flags, slot);
+  if (rc == TRI_ATTN_OK) ++h->ring_next;
+  return rc;
+}
+
+int tri_attn_host_wait(tri_attn_handle* h) {
+  if (!h) return TRI_ATTN_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+  const int rc = host_drain(h);
+  if (rc != TRI_ATTN_OK) return rc;
+  // every download follows the blocks that produced it, so the status word is
+  // final once copy_out has drained
+  return read_status(h, h->copy_out ? h->copy_out : nullptr);
 }
 
 int tri_attn_get_status(tri_attn_handle* h, void* stream) {
@@ -991,8 +1082,11 @@ int tri_attn_debug_workspace(tri_attn_handle* h, void** q, void** k, void** v, v
 int tri_attn_destroy(tri_attn_handle* h) {
   if (!h) return TRI_ATTN_OK;
   cudaSetDevice(h->device);
-  void* ptrs[] = {h->w_qkvg, h->w_g, h->w_o, h->w_b, h->gamma, h->beta, h->b_g,
-                  h->b_o,    h->status, h->ws, h->stage, h->stage_mask};
+  if (h->copy_in) cudaStreamSynchronize(h->copy_in);
+  if (h->copy_out) cudaStreamSynchronize(h->copy_out);
+  void* ptrs[] = {h->w_qkvg, h->w_g,  h->w_o,      h->w_b,      h->gamma,    h->beta,
+                  h->b_g,    h->b_o,  h->status,   h->ws,       h->stage[0], h->stage[1],
+                  h->stage[2], h->stage_mask};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   for (auto& vec : h->ev)
@@ -1001,9 +1095,13 @@ int tri_attn_destroy(tri_attn_handle* h) {
       if (p.b) cudaEventDestroy(p.b);
     }
   if (h->chunk_ev) cudaEventDestroy(h->chunk_ev);
+  if (h->up_ev) cudaEventDestroy(h->up_ev);
   for (cudaEvent_t e : h->in_ev)
     if (e) cudaEventDestroy(e);
-  if (h->copy_st) cudaStreamDestroy(h->copy_st);
+  for (cudaEvent_t e : h->slot_free)
+    if (e) cudaEventDestroy(e);
+  if (h->copy_in) cudaStreamDestroy(h->copy_in);
+  if (h->copy_out) cudaStreamDestroy(h->copy_out);
   delete h;
   return TRI_ATTN_OK;
 }
