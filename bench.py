@@ -65,7 +65,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--e2e-steps", type=int, default=8)
+    ap.add_argument("--e2e-steps", type=int, default=16)
     ap.add_argument("--workload", type=int, default=WORKLOAD,
                     help="workload index (the metric is quoted on the default; others are for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
