@@ -57,7 +57,7 @@ struct ProjArgs {
   const __nv_bfloat16* Z;
   const uint8_t* mask;
   int N, orient, row0, rows;
-  int write_qkvg, write_bias;
+  int write_qkv, write_bias;
   const uint8_t* w_img;  // [Wq; Wk; Wv] as the shared-memory image of the MMA B operand
   const float *w_b, *gamma, *beta;  // w_b pre-scaled by log2(e)
   float eps, q_scale;

@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int hc = (warp % 8) >> 2;               // channel half (LN) / output of a half (epilogue)
   const int p = wq * 32 + lane;                 // pair within the tile = TMEM lane
   const uint32_t bar_id = 1 + grp;
-  const bool qkvg = a.write_qkvg != 0;
+  const bool qkv = a.write_qkv != 0;
   uint8_t* sA = smem + kSmemA + grp * kATileBytes;
 
   for (int idx = tid; idx < kHeads * kCz; idx += kThreads)
@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && qkvg) {
+  if (warp == 0 && qkv) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot + static_cast<uint32_t>(grp * 256);
-  if (tid == 0 && qkvg) {
+  if (tid == 0 && qkv) {
     mbar_arrive_expect_tx(w_bar, kWImgBytes);
     for (uint32_t off = 0; off < kWImgBytes; off += 32768)
       bulk_load(smem + kSmemW + off, a.w_img + off, 32768, w_bar);
@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __float2bfloat16_rn(key_valid ? b : kMaskedLogit);
       }
     }
-    if (!qkvg) {
+    if (!qkv) {
       // bias only: the buffer (and the exchange area) is free once every
       // thread of the group has read them
       named_barrier_sync(bar_id, kGroupThreads);
@@ -386,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---- teardown: no copy may still be writing this CTA's smem
-  if (tid == 0 && qkvg && !w_ready) {
+  if (tid == 0 && qkv && !w_ready) {
     if (!mbar_wait(w_bar, 0, nullptr)) report_status(a.status, kStatusTimeout);
   }
   if (mma_thread && z_pending) {
@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0 && qkvg) {
+  if (warp == 0 && qkv) {
     tc_fence_after();
     tmem_dealloc(*tmem_slot, kTmemCols);
   }

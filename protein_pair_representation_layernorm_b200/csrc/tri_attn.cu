@@ -495,7 +495,7 @@ int forward_impl(tri_attn_handle* h, const void* Z, int N, const uint8_t* mask, 
     a.orient = orient;
     a.row0 = row0;
     a.rows = nrows;
-    a.write_qkvg = wq;
+    a.write_qkv = wq;
     a.write_bias = wb;
     a.w_img = static_cast<const uint8_t*>(h->w_qkvg);
     a.w_b = h->w_b;
