@@ -142,3 +142,12 @@ def test_attention_backward_rejects_bad_arguments_without_device():
     assert call(N=46341, workspace_bytes=ws_bytes(3, 46341)) == binding.TRI_ATTN_ERR_UNSUPPORTED
     if not torch.cuda.is_available():
         assert call() == binding.TRI_ATTN_ERR_NO_DEVICE
+
+
+def test_async_host_calls_reject_bad_arguments_without_device():
+    L = binding.lib()
+    buf = ctypes.c_void_p(0x10000)
+    orients = (ctypes.c_int * 2)(0, 1)
+    assert L.tri_attn_forward_host_async(None, buf, 16, None, orients, 2, buf, None, 0) == \
+        binding.TRI_ATTN_ERR_INVALID_ARG
+    assert L.tri_attn_host_wait(None) == binding.TRI_ATTN_ERR_INVALID_ARG

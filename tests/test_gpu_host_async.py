@@ -76,3 +76,22 @@ def test_pipelined_growing_problem_size():
     assert torch.equal(o1.view(torch.int16), _sync_ref(blk, small, [0, 1]).view(torch.int16))
     assert torch.equal(o2.view(torch.int16), _sync_ref(blk, big, [1, 0]).view(torch.int16))
     blk.close()
+
+
+def test_pipelined_calls_at_the_benchmark_size():
+    """N = 1536 (the benchmark's problem), four pipelined calls on two
+    alternating inputs: each result equals the synchronous call bit for bit."""
+    N = 1536
+    a = workloads.workload_inputs(3)
+    b = workloads.make_inputs(N, "bf16", 333)
+    b = workloads.Inputs(Z=b.Z, **{k: getattr(a, k) for k in (
+        "mask", "gamma", "beta", "Wq", "Wk", "Wv", "Wg", "bg", "Wb", "Wo", "bo")})
+    blk = block_for(a)
+    want = [_sync_ref(blk, p, [0, 1]) for p in (a, b)]
+    st = torch.cuda.Stream()
+    zs = [a.Z.clone().pin_memory(), b.Z.clone().pin_memory()]
+    outs = [blk.forward_host_async(zs[k % 2], [0, 1], a.mask, stream=st) for k in range(4)]
+    assert blk.host_wait() == binding.TRI_ATTN_OK
+    for k, got in enumerate(outs):
+        assert torch.equal(got.view(torch.int16), want[k % 2].view(torch.int16)), k
+    blk.close()
