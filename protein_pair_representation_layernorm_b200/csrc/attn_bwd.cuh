@@ -71,7 +71,7 @@ __device__ __forceinline__ void stage_rows(const float* blk, int k0, int N, floa
 }
 
 // ------------------------------------------------------------------ bwd_stats
-__global__ void __launch_bounds__(kThreadsRow) bwd_stats(BwdArgs a) {
+__global__ void __launch_bounds__(kThreadsRow, 4) bwd_stats(BwdArgs a) {
   __shared__ float sK[kTileK][kD], sV[kTileK][kD];
   __shared__ float sB[kThreadsRow][kTileK + 1];
   __shared__ unsigned char sM[kTileK];
@@ -189,7 +189,8 @@ __global__ void __launch_bounds__(kThreadsRow) bwd_dq(BwdArgs a) {
 }
 
 // ------------------------------------------------------------------- bwd_dkdv
-__global__ void __launch_bounds__(kThreadsRow) bwd_dkdv(BwdArgs a) {
+constexpr int kDkdvThreads = kThreadsRow;  // one thread per key
+__global__ void __launch_bounds__(kDkdvThreads) bwd_dkdv(BwdArgs a) {
   __shared__ float sQ[kTileJ][kD], sG[kTileJ][kD];
   __shared__ float sB[kTileJ][kThreadsRow];
   __shared__ float sL[kTileJ], sDj[kTileJ];
@@ -254,7 +255,7 @@ __global__ void __launch_bounds__(kThreadsRow) bwd_dkdv(BwdArgs a) {
 // (queries j0 + 4 (t / 16) + a, keys k0 + 4 (t % 16) + b).  Per row, the
 // row's q, dO, k, v rows of the block are staged transposed ([c][row], pitch
 // kTr) so that a thread reads its four rows' channel c as one float4.
-__global__ void __launch_bounds__(kBlkThreads) bwd_dbias(BwdArgs a) {
+__global__ void __launch_bounds__(kBlkThreads, 2) bwd_dbias(BwdArgs a) {
   __shared__ __align__(16) float sQ[kD][kTr], sG[kD][kTr], sK[kD][kTr], sV[kD][kTr];
   __shared__ float sL[kBlk], sDj[kBlk];
   const int h = blockIdx.z, j0 = blockIdx.y * kBlk, k0 = blockIdx.x * kBlk, t = threadIdx.x;

@@ -1321,7 +1321,7 @@ extern "C" int tri_attn_attention_backward(const float* Q, const float* K, const
   CUDA_TRY(cudaGetLastError());
   tri::bwd::bwd_dq<<<grid_rows, tri::bwd::kThreadsRow, 0, st>>>(a);
   CUDA_TRY(cudaGetLastError());
-  tri::bwd::bwd_dkdv<<<grid_rows, tri::bwd::kThreadsRow, 0, st>>>(a);
+  tri::bwd::bwd_dkdv<<<grid_rows, tri::bwd::kDkdvThreads, 0, st>>>(a);
   CUDA_TRY(cudaGetLastError());
   const unsigned blocks = static_cast<unsigned>((N + tri::bwd::kBlk - 1) / tri::bwd::kBlk);
   tri::bwd::bwd_dbias<<<dim3(blocks, blocks, tri::kHeads), tri::bwd::kBlkThreads, 0, st>>>(a);
