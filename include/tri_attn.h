@@ -294,6 +294,16 @@ int tri_attn_forward_noalloc(const tri_attn_params *params, const void *Z, int N
  * TRI_ATTN_ERR_NO_DEVICE, TRI_ATTN_ERR_CUDA (launch failure).
  * Flags: TRI_ATTN_FLAG_SYNC synchronises the stream before returning. */
 size_t tri_attn_attention_backward_workspace_bytes(int rows, int N);
+
+/* The forward of the same attention core (fp32), for training loops that pair
+ * it with tri_attn_attention_backward: writes o [rows][H][N][d] (16-byte
+ * aligned) and the natural-log log-sum-exp lse [rows][H][N] of each query's
+ * scores (+inf for a query whose every key is masked; its o is 0).  Same
+ * inputs, layouts and errors as the backward; one kernel launch (the backward's
+ * row-statistics kernel with o written out).  Flags: TRI_ATTN_FLAG_SYNC. */
+int tri_attn_attention_forward(const float *Q, const float *K, const float *V,
+                               const float *bias, const uint8_t *mask, int rows, int N,
+                               float *O, float *lse, void *stream, unsigned flags);
 int tri_attn_attention_backward(const float *Q, const float *K, const float *V,
                                 const float *bias, const uint8_t *mask, const float *dO,
                                 int rows, int N, float *dQ, float *dK, float *dV,

@@ -100,6 +100,7 @@ def lib() -> ctypes.CDLL:
         L.tri_attn_attention_backward_workspace_bytes.restype = sz
         L.tri_attn_attention_backward.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, vp, vp, vp, vp,
                                                   vp, sz, vp, cu]
+        L.tri_attn_attention_forward.argtypes = [vp, vp, vp, vp, vp, ci, ci, vp, vp, vp, cu]
         L.tri_attn_destroy.argtypes = [vp]
         L.tri_attn_status_string.argtypes = [ci]
         L.tri_attn_status_string.restype = ctypes.c_char_p
@@ -195,6 +196,13 @@ def tri_attn_forward_noalloc(params: tri_attn_params, Z_ptr, N: int, mask_ptr, o
 
 def tri_attn_destroy(h) -> int:
     return lib().tri_attn_destroy(h)
+
+
+def tri_attn_attention_forward(Q, K, V, bias, mask, rows: int, N: int, O, lse, stream=None,
+                               flags: int = 0) -> int:
+    """Forward of the attention core (device pointers); see tri_attn.h."""
+    return lib().tri_attn_attention_forward(Q, K, V, bias, mask, int(rows), int(N), O, lse,
+                                            stream, int(flags))
 
 
 def tri_attn_attention_backward_workspace_bytes(rows: int, N: int) -> int:
@@ -392,3 +400,48 @@ def attention_backward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, bias: 
     if rc != TRI_ATTN_OK:
         raise TriAttnError(rc, "tri_attn_attention_backward")
     return dQ, dK, dV, dB
+
+
+def _core_checked(Q, K, V, bias):
+    rows, H, N, d = Q.shape
+    for t in (Q, K, V):
+        if t.dtype != torch.float32 or not t.is_cuda or tuple(t.shape) != (rows, H, N, d):
+            raise ValueError("Q, K, V must be fp32 CUDA tensors of one shape [rows][H][N][d]")
+    if bias.dtype != torch.float32 or tuple(bias.shape) != (H, N, N):
+        raise ValueError("bias must be an fp32 CUDA tensor [H][N][N]")
+    return rows, N
+
+
+def attention_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, bias: torch.Tensor,
+                      mask: torch.Tensor | None = None, stream=None):
+    """(o, lse) of the attention core on the GPU (fp32; layouts as attention_backward)."""
+    rows, N = _core_checked(Q, K, V, bias)
+    Q, K, V, bias = (t.contiguous() for t in (Q, K, V, bias))
+    m = None if mask is None else mask.to(device=Q.device, dtype=torch.uint8).contiguous()
+    O = torch.empty_like(Q)
+    lse = torch.empty(Q.shape[:3], dtype=torch.float32, device=Q.device)
+    rc = tri_attn_attention_forward(_ptr(Q), _ptr(K), _ptr(V), _ptr(bias), _ptr(m), rows, N,
+                                    _ptr(O), _ptr(lse), _stream_handle(stream), 0)
+    if rc != TRI_ATTN_OK:
+        raise TriAttnError(rc, "tri_attn_attention_forward")
+    return O, lse
+
+
+class AttentionCore(torch.autograd.Function):
+    """The attention core as a differentiable torch op on the library's fp32
+    kernels: o = softmax_k(q . k / sqrt(d) + bias, masked) v per problem row,
+    with gradients for q, k, v and the (row-shared) bias.  Call as
+    AttentionCore.apply(Q, K, V, bias, mask)."""
+
+    @staticmethod
+    def forward(ctx, Q, K, V, bias, mask=None):
+        O, _ = attention_forward(Q, K, V, bias, mask)
+        ctx.save_for_backward(Q, K, V, bias)
+        ctx.mask = mask
+        return O
+
+    @staticmethod
+    def backward(ctx, dO):
+        Q, K, V, bias = ctx.saved_tensors
+        dQ, dK, dV, dB = attention_backward(Q, K, V, bias, dO.contiguous(), ctx.mask)
+        return dQ, dK, dV, dB, None

@@ -12,7 +12,8 @@
 // p is recomputed from the row statistics instead of being stored: an R x N x N
 // x H probability tensor would not fit (58 GB at N = 1536).  Four kernels:
 //   bwd_stats   thread = query: one pass over the keys with a running maximum
-//               gives LSE_j = log sum_k exp(s_jk) and D_j;
+//               gives LSE_j = log sum_k exp(s_jk) and D_j (alone, with o written
+//               out, it is also the forward of the core);
 //   bwd_dq      thread = query: dQ_j, keys streamed through shared memory;
 //   bwd_dkdv    thread = key: dK_k and dV_k, queries streamed through shared
 //               memory;
@@ -28,10 +29,11 @@ namespace tri {
 namespace bwd {
 
 struct BwdArgs {
-  const float *Q, *K, *V, *B, *dO;  // [rows][H][N][d]; B: [H][N][N]
+  const float *Q, *K, *V, *B, *dO;  // [rows][H][N][d]; B: [H][N][N]; dO may be null (forward)
   const uint8_t* mask;              // [N] or nullptr
   float *dQ, *dK, *dV, *dB;         // like Q, K, V and B
-  float *lse, *D;                   // [rows][H][N] scratch
+  float *lse, *D;                   // [rows][H][N] scratch (D unused without dO)
+  float* O;                         // [rows][H][N][d]: o written here when not null
   int rows, N;
 };
 
@@ -123,14 +125,24 @@ __global__ void __launch_bounds__(kThreadsRow, 4) bwd_stats(BwdArgs a) {
     m = mn;
   }
   if (!jv) return;
-  float g[kD];
-  load_vec(a.dO + (blk + j) * kD, g);
-  float dd = 0.f;
-#pragma unroll
-  for (int c = 0; c < kD; ++c) dd = fmaf(g[c], o[c], dd);
   // a query with every key masked: LSE = +inf makes every p exactly 0
   a.lse[blk + j] = l > 0.f ? m + logf(l) : INFINITY;
-  a.D[blk + j] = l > 0.f ? dd / l : 0.f;
+  const float inv = l > 0.f ? 1.0f / l : 0.f;
+  if (a.O) {  // the forward: o = O / l
+    float4* dst = reinterpret_cast<float4*>(a.O + (blk + j) * kD);
+#pragma unroll
+    for (int c = 0; c < kD / 4; ++c)
+      dst[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv,
+                           o[4 * c + 3] * inv);
+  }
+  if (a.dO) {
+    float g[kD];
+    load_vec(a.dO + (blk + j) * kD, g);
+    float dd = 0.f;
+#pragma unroll
+    for (int c = 0; c < kD; ++c) dd = fmaf(g[c], o[c], dd);
+    a.D[blk + j] = dd * inv;
+  }
 }
 
 // --------------------------------------------------------------------- bwd_dq

@@ -1283,6 +1283,36 @@ extern "C" size_t tri_attn_attention_backward_workspace_bytes(int rows, int N) {
   return 2 * static_cast<size_t>(rows) * tri::kHeads * N * sizeof(float);
 }
 
+extern "C" int tri_attn_attention_forward(const float* Q, const float* K, const float* V,
+                                          const float* bias, const uint8_t* mask, int rows,
+                                          int N, float* O, float* lse, void* stream,
+                                          unsigned flags) {
+  const void* vec[] = {Q, K, V, O};
+  for (const void* ptr : vec)
+    if (!ptr || reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return TRI_ATTN_ERR_INVALID_ARG;
+  if (!bias || !lse || rows < 1 || N < 1) return TRI_ATTN_ERR_INVALID_ARG;
+  if (rows > 65535 || N > 46340) return TRI_ATTN_ERR_UNSUPPORTED;
+  int rc = check_device();
+  if (rc != TRI_ATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  tri::bwd::BwdArgs a{};
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.B = bias;
+  a.mask = mask;
+  a.lse = lse;
+  a.O = O;
+  a.rows = rows;
+  a.N = N;
+  const unsigned tiles = static_cast<unsigned>((N + tri::bwd::kThreadsRow - 1) / tri::bwd::kThreadsRow);
+  tri::bwd::bwd_stats<<<dim3(tiles, static_cast<unsigned>(rows), tri::kHeads),
+                        tri::bwd::kThreadsRow, 0, st>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  if (flags & TRI_ATTN_FLAG_SYNC) CUDA_TRY(cudaStreamSynchronize(st));
+  return TRI_ATTN_OK;
+}
+
 extern "C" int tri_attn_attention_backward(const float* Q, const float* K, const float* V,
                                            const float* bias, const uint8_t* mask,
                                            const float* dO, int rows, int N, float* dQ,

@@ -151,3 +151,21 @@ def test_async_host_calls_reject_bad_arguments_without_device():
     assert L.tri_attn_forward_host_async(None, buf, 16, None, orients, 2, buf, None, 0) == \
         binding.TRI_ATTN_ERR_INVALID_ARG
     assert L.tri_attn_host_wait(None) == binding.TRI_ATTN_ERR_INVALID_ARG
+
+
+def test_core_forward_rejects_bad_arguments_without_device():
+    L = binding.lib()
+    buf = 0x10000
+    ok = dict(Q=buf, K=buf, V=buf, bias=buf, mask=None, rows=2, N=40, O=buf, lse=buf,
+              stream=None, flags=0)
+
+    def call(**kw):
+        return L.tri_attn_attention_forward(*dict(ok, **kw).values())
+
+    assert call(Q=None) == binding.TRI_ATTN_ERR_INVALID_ARG
+    assert call(O=buf + 8) == binding.TRI_ATTN_ERR_INVALID_ARG
+    assert call(lse=None) == binding.TRI_ATTN_ERR_INVALID_ARG
+    assert call(N=0) == binding.TRI_ATTN_ERR_INVALID_ARG
+    assert call(rows=70000) == binding.TRI_ATTN_ERR_UNSUPPORTED
+    if not torch.cuda.is_available():
+        assert call() == binding.TRI_ATTN_ERR_NO_DEVICE

@@ -102,3 +102,37 @@ def test_backward_at_n768_sampled_rows_and_jacobian_property():
     assert float(np.abs(sums).max()) <= 1e-4 * float(np.abs(db).max()) * np.sqrt(N)
     # masked keys receive no bias gradient
     assert not np.any(db[:, :, mask == 0])
+
+
+@pytest.mark.parametrize("rows,N,mask_kind,seed", [(3, 70, None, 11), (2, 133, "random", 12),
+                                                   (1, 40, "all", 13)])
+def test_core_forward_matches_oracle(rows, N, mask_kind, seed):
+    q, k, v, g, bias, mask = _inputs(seed, rows, N, mask_kind)
+    T = lambda a: torch.from_numpy(a).cuda()  # noqa: E731
+    o, lse = binding.attention_forward(T(q), T(k), T(v), T(bias),
+                                       None if mask is None else T(mask))
+    torch.cuda.synchronize()
+    o = o.cpu().numpy().astype(np.float64)
+    for r in range(rows):
+        ref = oracle.attend(_to_oracle(q[r:r + 1])[0], _to_oracle(k[r:r + 1])[0],
+                            _to_oracle(v[r:r + 1])[0], bias.astype(np.float64), mask)
+        _check(f"core forward N={N} row {r} mask={mask_kind}", _to_oracle(o[r:r + 1])[0], ref)
+    if mask_kind == "all":
+        assert torch.isinf(lse).all() and (lse > 0).all()
+
+
+def test_autograd_function_gives_the_oracle_gradients():
+    """AttentionCore.apply inside a torch graph: a scalar loss that weights o
+    by a fixed tensor G has d loss / d o = G, so every input's gradient must be
+    the oracle's gradient for dout = G."""
+    q, k, v, g, bias, mask = _inputs(14, 2, 90, "random")
+    T = lambda a: torch.from_numpy(a).cuda().requires_grad_()  # noqa: E731
+    tq, tk, tv, tb = T(q), T(k), T(v), T(bias)
+    o = binding.AttentionCore.apply(tq, tk, tv, tb, torch.from_numpy(mask).cuda())
+    (o * torch.from_numpy(g).cuda()).sum().backward()
+    rq, rk, rv, rb = oracle.tri_attn_core_bwd(_to_oracle(q), _to_oracle(k), _to_oracle(v),
+                                              bias.astype(np.float64), _to_oracle(g), mask)
+    _check("autograd dQ", _to_oracle(tq.grad.cpu().numpy().astype(np.float64)), rq)
+    _check("autograd dK", _to_oracle(tk.grad.cpu().numpy().astype(np.float64)), rk)
+    _check("autograd dV", _to_oracle(tv.grad.cpu().numpy().astype(np.float64)), rv)
+    _check("autograd dbias", tb.grad.cpu().numpy().astype(np.float64), rb)
