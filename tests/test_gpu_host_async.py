@@ -95,3 +95,20 @@ def test_pipelined_calls_at_the_benchmark_size():
     for k, got in enumerate(outs):
         assert torch.equal(got.view(torch.int16), want[k % 2].view(torch.int16)), k
     blk.close()
+
+
+def test_pipelined_calls_on_an_fp32_handle():
+    """fp32 handles upload Z whole (no piecewise projection) and run the SIMT
+    kernels; pipelined calls must still equal synchronous ones bit for bit."""
+    N = 70
+    inp = workloads.make_inputs(N, "f32", 340, "random:0.1")
+    blk = block_for(inp)
+    st = torch.cuda.Stream()
+    zs = [inp.Z.clone().pin_memory() for _ in range(4)]
+    orients = [[0, 1], [1], [1, 0], [0]]
+    outs = [blk.forward_host_async(z, o, inp.mask, stream=st) for z, o in zip(zs, orients)]
+    assert blk.host_wait() == binding.TRI_ATTN_OK
+    for got, o in zip(outs, orients):
+        want = _sync_ref(blk, inp, o)
+        assert torch.equal(got.view(torch.int32), want.view(torch.int32))
+    blk.close()
