@@ -310,6 +310,53 @@ int tri_attn_attention_backward(const float *Q, const float *K, const float *V,
                                 float *dbias, void *workspace, size_t workspace_bytes,
                                 void *stream, unsigned flags);
 
+/* ---- the same attention core on the tensor cores (bf16 operands) ---------
+ *
+ * The mathematics, layouts and natural units of the two fp32 calls above, with
+ * bf16 operands: Q, K, V, O, dO bf16 [rows][H][N][d] (H = 4, d = 32), bias
+ * bf16 [H][N][N], mask uint8 [N] (1 = valid key) or NULL.  Products run on
+ * tcgen05 tensor cores in bf16 with fp32 accumulation: q * log2(e)/sqrt(d),
+ * the bias in base 2, and the probabilities and ds_jk fed to the gradient
+ * products are rounded to bf16 (relative 2^-9 each); lse, the row statistics
+ * and every sum are fp32.
+ *
+ * `workspace` (16-byte aligned, at least
+ * tri_attn_attention_bf16_workspace_bytes(rows, N) bytes, caller-owned, the
+ * same size for both calls) holds the device status word, the scaled q, the
+ * padded base-2 bias (and its transpose) and the per-query statistics.  Both
+ * calls are asynchronous on `stream`; with TRI_ATTN_FLAG_SYNC they wait and
+ * return the device status (TRI_ATTN_ERR_TIMEOUT if a kernel's bounded wait
+ * expired).  The calls allocate nothing.
+ * Errors: TRI_ATTN_ERR_INVALID_ARG (NULL or misaligned pointer: Q, K, V, O,
+ * dO, dQ, dK, dV, dbias and workspace must be 16-byte aligned, lse 4-byte;
+ * rows or N < 1; workspace too small), TRI_ATTN_ERR_UNSUPPORTED (rows > 65535
+ * or N > 46340), TRI_ATTN_ERR_NO_DEVICE, TRI_ATTN_ERR_CUDA (launch failure). */
+size_t tri_attn_attention_bf16_workspace_bytes(int rows, int N);
+
+/* o (bf16) and lse (fp32 [rows][H][N], natural log, +inf for a query whose
+ * every key is masked; its o is 0) — the flash-style forward kernel of the
+ * block (tri_attn_fwd, scores never in memory) run on the caller's Q, K, V
+ * and bias, after two preparation kernels (q scaled; the bias in base 2 with
+ * the mask folded in).  lse may be NULL. */
+int tri_attn_attention_forward_bf16(const void *Q, const void *K, const void *V,
+                                    const void *bias, const uint8_t *mask, int rows, int N,
+                                    void *O, float *lse, void *workspace,
+                                    size_t workspace_bytes, void *stream, unsigned flags);
+
+/* Gradients dQ, dK, dV (fp32 [rows][H][N][d]) and dbias (fp32 [H][N][N],
+ * summed over the rows) from the operands, the forward's o and lse (those of
+ * tri_attn_attention_forward_bf16 on the same operands) and dO.  Five kernel
+ * launches after the preparation: dQ (a CTA per 3 rows x 128 queries x head,
+ * walking the keys), dK and dV (per 2 rows x 128 keys x head, walking the
+ * queries), dbias (per 128 queries x 64 keys x head, walking every row, so it
+ * is written once per element: no atomics, deterministic). */
+int tri_attn_attention_backward_bf16(const void *Q, const void *K, const void *V,
+                                     const void *bias, const uint8_t *mask, const void *O,
+                                     const float *lse, const void *dO, int rows, int N,
+                                     float *dQ, float *dK, float *dV, float *dbias,
+                                     void *workspace, size_t workspace_bytes, void *stream,
+                                     unsigned flags);
+
 /* Release everything the handle owns.  NULL-safe.  Not stream-ordered:
  * call it after the work that uses the handle has completed. */
 int tri_attn_destroy(tri_attn_handle *h);

@@ -101,6 +101,12 @@ def lib() -> ctypes.CDLL:
         L.tri_attn_attention_backward.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, vp, vp, vp, vp,
                                                   vp, sz, vp, cu]
         L.tri_attn_attention_forward.argtypes = [vp, vp, vp, vp, vp, ci, ci, vp, vp, vp, cu]
+        L.tri_attn_attention_bf16_workspace_bytes.argtypes = [ci, ci]
+        L.tri_attn_attention_bf16_workspace_bytes.restype = sz
+        L.tri_attn_attention_forward_bf16.argtypes = [vp, vp, vp, vp, vp, ci, ci, vp, vp, vp, sz,
+                                                      vp, cu]
+        L.tri_attn_attention_backward_bf16.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, vp,
+                                                       vp, vp, vp, vp, sz, vp, cu]
         L.tri_attn_destroy.argtypes = [vp]
         L.tri_attn_status_string.argtypes = [ci]
         L.tri_attn_status_string.restype = ctypes.c_char_p
@@ -203,6 +209,27 @@ def tri_attn_attention_forward(Q, K, V, bias, mask, rows: int, N: int, O, lse, s
     """Forward of the attention core (device pointers); see tri_attn.h."""
     return lib().tri_attn_attention_forward(Q, K, V, bias, mask, int(rows), int(N), O, lse,
                                             stream, int(flags))
+
+
+def tri_attn_attention_bf16_workspace_bytes(rows: int, N: int) -> int:
+    return int(lib().tri_attn_attention_bf16_workspace_bytes(int(rows), int(N)))
+
+
+def tri_attn_attention_forward_bf16(Q, K, V, bias, mask, rows: int, N: int, O, lse, workspace,
+                                    workspace_bytes: int, stream=None, flags: int = 0) -> int:
+    """Tensor-core forward of the attention core (device pointers); see tri_attn.h."""
+    return lib().tri_attn_attention_forward_bf16(Q, K, V, bias, mask, int(rows), int(N), O, lse,
+                                                 workspace, int(workspace_bytes), stream,
+                                                 int(flags))
+
+
+def tri_attn_attention_backward_bf16(Q, K, V, bias, mask, O, lse, dO, rows: int, N: int, dQ, dK,
+                                     dV, dbias, workspace, workspace_bytes: int, stream=None,
+                                     flags: int = 0) -> int:
+    """Tensor-core backward of the attention core (device pointers); see tri_attn.h."""
+    return lib().tri_attn_attention_backward_bf16(Q, K, V, bias, mask, O, lse, dO, int(rows),
+                                                  int(N), dQ, dK, dV, dbias, workspace,
+                                                  int(workspace_bytes), stream, int(flags))
 
 
 def tri_attn_attention_backward_workspace_bytes(rows: int, N: int) -> int:
@@ -427,21 +454,90 @@ def attention_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, bias: t
     return O, lse
 
 
+def _core_checked_bf16(Q, K, V, bias, *more):
+    rows, H, N, d = Q.shape
+    for t in (Q, K, V) + more:
+        if t.dtype != torch.bfloat16 or not t.is_cuda or tuple(t.shape) != (rows, H, N, d):
+            raise ValueError("Q, K, V (O, dO) must be bf16 CUDA tensors of one shape "
+                             "[rows][H][N][d]")
+    if bias.dtype != torch.bfloat16 or tuple(bias.shape) != (H, N, N):
+        raise ValueError("bias must be a bf16 CUDA tensor [H][N][N]")
+    return rows, N
+
+
+def _core_workspace(rows, N, device):
+    nbytes = tri_attn_attention_bf16_workspace_bytes(rows, N)
+    return torch.empty((nbytes + 15) // 16 * 4, dtype=torch.float32, device=device), nbytes
+
+
+def attention_forward_bf16(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, bias: torch.Tensor,
+                           mask: torch.Tensor | None = None, stream=None):
+    """(o, lse) of the attention core on the tensor cores: bf16 Q, K, V
+    [rows][H][N][d] and bias [H][N][N] (natural-unit logits), o bf16, lse fp32
+    [rows][H][N] (natural log; +inf for a query whose every key is masked)."""
+    rows, N = _core_checked_bf16(Q, K, V, bias)
+    Q, K, V, bias = (t.contiguous() for t in (Q, K, V, bias))
+    m = None if mask is None else mask.to(device=Q.device, dtype=torch.uint8).contiguous()
+    O = torch.empty_like(Q)
+    lse = torch.empty(Q.shape[:3], dtype=torch.float32, device=Q.device)
+    ws, nbytes = _core_workspace(rows, N, Q.device)
+    rc = tri_attn_attention_forward_bf16(_ptr(Q), _ptr(K), _ptr(V), _ptr(bias), _ptr(m), rows, N,
+                                         _ptr(O), _ptr(lse), _ptr(ws), nbytes,
+                                         _stream_handle(stream), 0)
+    if rc != TRI_ATTN_OK:
+        raise TriAttnError(rc, "tri_attn_attention_forward_bf16")
+    return O, lse
+
+
+def attention_backward_bf16(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, bias: torch.Tensor,
+                            O: torch.Tensor, lse: torch.Tensor, dO: torch.Tensor,
+                            mask: torch.Tensor | None = None, stream=None, sync: bool = False):
+    """Gradients (dQ, dK, dV, dbias), fp32, of the attention core on the tensor
+    cores, from the bf16 operands, the forward's o (bf16) and lse (fp32) and
+    the bf16 dO.  With sync, waits and raises on a device-side timeout."""
+    rows, N = _core_checked_bf16(Q, K, V, bias, O, dO)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != tuple(Q.shape[:3]):
+        raise ValueError("lse must be an fp32 CUDA tensor [rows][H][N]")
+    Q, K, V, bias, O, lse, dO = (t.contiguous() for t in (Q, K, V, bias, O, lse, dO))
+    m = None if mask is None else mask.to(device=Q.device, dtype=torch.uint8).contiguous()
+    dQ = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    dK, dV = torch.empty_like(dQ), torch.empty_like(dQ)
+    dB = torch.empty(bias.shape, dtype=torch.float32, device=Q.device)
+    ws, nbytes = _core_workspace(rows, N, Q.device)
+    rc = tri_attn_attention_backward_bf16(_ptr(Q), _ptr(K), _ptr(V), _ptr(bias), _ptr(m),
+                                          _ptr(O), _ptr(lse), _ptr(dO), rows, N, _ptr(dQ),
+                                          _ptr(dK), _ptr(dV), _ptr(dB), _ptr(ws), nbytes,
+                                          _stream_handle(stream), TRI_ATTN_FLAG_SYNC if sync else 0)
+    if rc != TRI_ATTN_OK:
+        raise TriAttnError(rc, "tri_attn_attention_backward_bf16")
+    return dQ, dK, dV, dB
+
+
 class AttentionCore(torch.autograd.Function):
-    """The attention core as a differentiable torch op on the library's fp32
-    kernels: o = softmax_k(q . k / sqrt(d) + bias, masked) v per problem row,
-    with gradients for q, k, v and the (row-shared) bias.  Call as
-    AttentionCore.apply(Q, K, V, bias, mask)."""
+    """The attention core as a differentiable torch op: o = softmax_k(q . k /
+    sqrt(d) + bias, masked) v per problem row, with gradients for q, k, v and
+    the (row-shared) bias.  fp32 inputs run the library's fp32 SIMT kernels;
+    bf16 inputs run the tensor-core forward and backward (gradients returned in
+    bf16, computed in fp32).  Call as AttentionCore.apply(Q, K, V, bias, mask)."""
 
     @staticmethod
     def forward(ctx, Q, K, V, bias, mask=None):
-        O, _ = attention_forward(Q, K, V, bias, mask)
-        ctx.save_for_backward(Q, K, V, bias)
+        if Q.dtype == torch.bfloat16:
+            O, lse = attention_forward_bf16(Q, K, V, bias, mask)
+            ctx.save_for_backward(Q, K, V, bias, O, lse)
+        else:
+            O, _ = attention_forward(Q, K, V, bias, mask)
+            ctx.save_for_backward(Q, K, V, bias)
         ctx.mask = mask
         return O
 
     @staticmethod
     def backward(ctx, dO):
+        if len(ctx.saved_tensors) == 6:
+            Q, K, V, bias, O, lse = ctx.saved_tensors
+            grads = attention_backward_bf16(Q, K, V, bias, O, lse,
+                                            dO.to(torch.bfloat16).contiguous(), ctx.mask)
+            return tuple(g.to(torch.bfloat16) for g in grads) + (None,)
         Q, K, V, bias = ctx.saved_tensors
         dQ, dK, dV, dB = attention_backward(Q, K, V, bias, dO.contiguous(), ctx.mask)
         return dQ, dK, dV, dB, None

@@ -72,6 +72,7 @@ struct ProjArgs {
 
 struct AttnArgs {
   __nv_bfloat16* O;  // [rows][H][N][d]
+  float* lse;        // [rows][H][N]: each query's natural-log log-sum-exp, or nullptr
   int N, rows;
   int debug_stall;
   int* status;

@@ -6,7 +6,8 @@
 //   tri_attn_fwd  (online-softmax attention, tcgen05 + TMA)     tensor/ALU-bound
 //   gate_out      (gate * o, output projection, residual)       HBM-bound
 // (fp32 handles run the SIMT kernels of kernels_f32.cuh instead; the backward
-// pass of the attention core runs the kernels of attn_bwd.cuh).  The logit
+// pass of the attention core runs the kernels of attn_bwd.cuh in fp32, or those
+// of attn_bwd_tc.cuh on the tensor cores for bf16 operands).  The logit
 // bias of every pair is needed by every row, so it is produced for all pairs
 // before any attention runs; when the workspace for all rows exceeds the
 // handle's limit, a bias-only pass runs first and the rest proceeds in row
@@ -27,6 +28,7 @@
 #include <vector>
 
 #include "attn_bwd.cuh"
+#include "attn_bwd_tc.cuh"
 #include "common.cuh"
 #include "gate_out.cuh"
 #include "kernels_f32.cuh"
@@ -181,6 +183,14 @@ int set_kernel_attrs() {
                                 tri::attn::kSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(tri::gout::gate_out, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 tri::gout::kSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(tri::bwdtc::bwd_rows<tri::bwdtc::kDQ>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                tri::bwdtc::RowsLayout<tri::bwdtc::kDQ>::kSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(tri::bwdtc::bwd_rows<tri::bwdtc::kDKDV>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                tri::bwdtc::RowsLayout<tri::bwdtc::kDKDV>::kSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(tri::bwdtc::bwd_dbias_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                tri::bwdtc::kDbSmemBytes));
   if (log_enabled()) {
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, tri::attn::tri_attn_fwd) == cudaSuccess)
@@ -1358,4 +1368,212 @@ extern "C" int tri_attn_attention_backward(const float* Q, const float* K, const
   CUDA_TRY(cudaGetLastError());
   if (flags & TRI_ATTN_FLAG_SYNC) CUDA_TRY(cudaStreamSynchronize(st));
   return TRI_ATTN_OK;
+}
+
+// ------------------------------------------------------------------ bf16 attention core
+namespace {
+
+struct CoreWs {
+  int* status = nullptr;
+  bf16 *qs = nullptr, *b2 = nullptr, *b2T = nullptr;
+  float *nlse2 = nullptr, *nD = nullptr;
+};
+
+// Workspace of the bf16 core calls: the device status word, Qs [rows][H][N][d]
+// bf16, b2 and b2T [H][N][ld] bf16, -lse2 and -D [rows][H][ld] fp32 (ld = N
+// rounded up to 128), each part 256-byte aligned.  Returns the bytes needed;
+// fills *w when base is set.
+size_t core_ws_layout(int rows, int N, void* base, CoreWs* w) {
+  const size_t ld = static_cast<size_t>(tri::bwdtc::padded_ld(N));
+  const size_t rh = static_cast<size_t>(rows) * tri::kHeads;
+  const size_t parts[6] = {sizeof(int), rh * N * tri::kD * 2, tri::kHeads * N * ld * 2,
+                           tri::kHeads * N * ld * 2, rh * ld * 4, rh * ld * 4};
+  size_t off[6], total = 0;
+  for (int p = 0; p < 6; ++p) {
+    off[p] = total;
+    total = align_up(total + parts[p], 256);
+  }
+  if (base != nullptr && w != nullptr) {
+    char* b = static_cast<char*>(base);
+    w->status = reinterpret_cast<int*>(b + off[0]);
+    w->qs = reinterpret_cast<bf16*>(b + off[1]);
+    w->b2 = reinterpret_cast<bf16*>(b + off[2]);
+    w->b2T = reinterpret_cast<bf16*>(b + off[3]);
+    w->nlse2 = reinterpret_cast<float*>(b + off[4]);
+    w->nD = reinterpret_cast<float*>(b + off[5]);
+  }
+  return total;
+}
+
+// [rows][H][N][d] bf16 operand, boxes of `box` rows x 32 (64-byte swizzle)
+bool operand_map(CUtensorMap* m, const void* p, int rows, int N, uint32_t box) {
+  return make_map_3d(m, p, tri::kD, N, static_cast<uint64_t>(rows) * tri::kHeads, tri::kD * 2,
+                     static_cast<uint64_t>(N) * tri::kD * 2, tri::kD, box,
+                     CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+// [H][N][ld] bf16 bias, boxes of 128 rows x 64 columns (128-byte swizzle)
+bool bias_map(CUtensorMap* m, const void* p, int N, int ld) {
+  return make_map_3d(m, p, ld, N, tri::kHeads, static_cast<uint64_t>(ld) * 2,
+                     static_cast<uint64_t>(N) * ld * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+int core_args_ok(const void* const* aligned16, int n, const void* bias, int rows, int N,
+                 void* workspace, size_t workspace_bytes) {
+  for (int i = 0; i < n; ++i)
+    if (!aligned16[i] || reinterpret_cast<uintptr_t>(aligned16[i]) % 16 != 0)
+      return TRI_ATTN_ERR_INVALID_ARG;
+  if (!bias || rows < 1 || N < 1) return TRI_ATTN_ERR_INVALID_ARG;
+  if (rows > 65535 || N > 46340) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 16 != 0 ||
+      workspace_bytes < core_ws_layout(rows, N, nullptr, nullptr))
+    return TRI_ATTN_ERR_INVALID_ARG;
+  return TRI_ATTN_OK;
+}
+
+// Clear the status word; Qs, b2 (and b2T when asked) from the caller's operands
+int core_prep(const void* Q, const void* bias, const uint8_t* mask, int rows, int N,
+              const CoreWs& w, bool transpose, cudaStream_t st) {
+  CUDA_TRY(cudaMemsetAsync(w.status, 0, sizeof(int), st));
+  const int ld = tri::bwdtc::padded_ld(N);
+  const long long n8 = static_cast<long long>(rows) * tri::kHeads * N * tri::kD / 8;
+  const int blocks = static_cast<int>(std::min<long long>((n8 + 255) / 256, 148 * 16));
+  tri::bwdtc::prep_q<<<blocks, 256, 0, st>>>(static_cast<const bf16*>(Q), w.qs, n8);
+  CUDA_TRY(cudaGetLastError());
+  tri::bwdtc::prep_bias<<<dim3(ld / 32, ld / 32, tri::kHeads), dim3(32, 8), 0, st>>>(
+      static_cast<const bf16*>(bias), mask, N, ld, w.b2, transpose ? w.b2T : nullptr);
+  CUDA_TRY(cudaGetLastError());
+  return TRI_ATTN_OK;
+}
+
+// With TRI_ATTN_FLAG_SYNC: wait for the call and return its device status.
+int core_finish(const CoreWs& w, cudaStream_t st, unsigned flags) {
+  if (!(flags & TRI_ATTN_FLAG_SYNC)) return TRI_ATTN_OK;
+  int s = 0;
+  CUDA_TRY(cudaMemcpyAsync(&s, w.status, sizeof(int), cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaStreamSynchronize(st));
+  return s;
+}
+
+}  // namespace
+
+extern "C" size_t tri_attn_attention_bf16_workspace_bytes(int rows, int N) {
+  if (rows < 1 || N < 1) return 0;
+  return core_ws_layout(rows, N, nullptr, nullptr);
+}
+
+extern "C" int tri_attn_attention_forward_bf16(const void* Q, const void* K, const void* V,
+                                               const void* bias, const uint8_t* mask, int rows,
+                                               int N, void* O, float* lse, void* workspace,
+                                               size_t workspace_bytes, void* stream,
+                                               unsigned flags) {
+  const void* vec[] = {Q, K, V, O};
+  int rc = core_args_ok(vec, 4, bias, rows, N, workspace, workspace_bytes);
+  if (rc != TRI_ATTN_OK) return rc;
+  if (lse && reinterpret_cast<uintptr_t>(lse) % 4 != 0) return TRI_ATTN_ERR_INVALID_ARG;
+  rc = check_device();
+  if (rc != TRI_ATTN_OK) return rc;
+  rc = set_kernel_attrs();
+  if (rc != TRI_ATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CoreWs w;
+  core_ws_layout(rows, N, workspace, &w);
+  rc = core_prep(Q, bias, mask, rows, N, w, false, st);
+  if (rc != TRI_ATTN_OK) return rc;
+  const int ld = tri::bwdtc::padded_ld(N);
+  CUtensorMap mq, mk, mv, mb;
+  if (!operand_map(&mq, w.qs, rows, N, tri::attn::kBJ) ||
+      !operand_map(&mk, K, rows, N, tri::attn::kBK) ||
+      !operand_map(&mv, V, rows, N, tri::attn::kBK) || !bias_map(&mb, w.b2, N, ld))
+    return TRI_ATTN_ERR_CUDA;
+  tri::AttnArgs a{};
+  a.O = static_cast<bf16*>(O);
+  a.lse = lse;
+  a.N = N;
+  a.rows = rows;
+  a.status = w.status;
+  const dim3 grid((N + tri::attn::kBJ - 1) / tri::attn::kBJ,
+                  (rows + tri::attn::kRows - 1) / tri::attn::kRows, tri::kHeads);
+  tri::attn::tri_attn_fwd<<<grid, tri::attn::kThreads, tri::attn::kSmemBytes, st>>>(mq, mk, mv,
+                                                                                 mb, a);
+  CUDA_TRY(cudaGetLastError());
+  return core_finish(w, st, flags);
+}
+
+extern "C" int tri_attn_attention_backward_bf16(const void* Q, const void* K, const void* V,
+                                                const void* bias, const uint8_t* mask,
+                                                const void* O, const float* lse, const void* dO,
+                                                int rows, int N, float* dQ, float* dK, float* dV,
+                                                float* dbias, void* workspace,
+                                                size_t workspace_bytes, void* stream,
+                                                unsigned flags) {
+  const void* vec[] = {Q, K, V, O, dO, dQ, dK, dV, dbias};
+  int rc = core_args_ok(vec, 9, bias, rows, N, workspace, workspace_bytes);
+  if (rc != TRI_ATTN_OK) return rc;
+  if (!lse || reinterpret_cast<uintptr_t>(lse) % 4 != 0) return TRI_ATTN_ERR_INVALID_ARG;
+  rc = check_device();
+  if (rc != TRI_ATTN_OK) return rc;
+  rc = set_kernel_attrs();
+  if (rc != TRI_ATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CoreWs w;
+  core_ws_layout(rows, N, workspace, &w);
+  rc = core_prep(Q, bias, mask, rows, N, w, true, st);
+  if (rc != TRI_ATTN_OK) return rc;
+  const int ld = tri::bwdtc::padded_ld(N);
+  {
+    const long long rh = static_cast<long long>(rows) * tri::kHeads;
+    const int blocks = static_cast<int>(std::min<long long>((rh * ld + 255) / 256, 148 * 16));
+    tri::bwdtc::prep_rows<<<blocks, 256, 0, st>>>(static_cast<const bf16*>(O),
+                                                  static_cast<const bf16*>(dO), lse, rh, N, ld,
+                                                  w.nlse2, w.nD);
+    CUDA_TRY(cudaGetLastError());
+  }
+  CUtensorMap q128, o128, k128, v128, q64, o64, k64, v64, mb, mbT;
+  if (!operand_map(&q128, w.qs, rows, N, 128) || !operand_map(&o128, dO, rows, N, 128) ||
+      !operand_map(&k128, K, rows, N, 128) || !operand_map(&v128, V, rows, N, 128) ||
+      !operand_map(&q64, w.qs, rows, N, 64) || !operand_map(&o64, dO, rows, N, 64) ||
+      !operand_map(&k64, K, rows, N, 64) || !operand_map(&v64, V, rows, N, 64) ||
+      !bias_map(&mb, w.b2, N, ld) || !bias_map(&mbT, w.b2T, N, ld))
+    return TRI_ATTN_ERR_CUDA;
+  namespace bt = tri::bwdtc;
+  bt::RowsArgs ra{};
+  ra.nlse2 = w.nlse2;
+  ra.nD = w.nD;
+  ra.N = N;
+  ra.rows = rows;
+  ra.ld = ld;
+  ra.status = w.status;
+  const unsigned mtiles = static_cast<unsigned>((N + bt::kTM - 1) / bt::kTM);
+  {
+    using L = bt::RowsLayout<bt::kDQ>;
+    ra.out1 = dQ;
+    ra.out2 = nullptr;
+    const dim3 grid(mtiles, (rows + L::kR - 1) / L::kR, tri::kHeads);
+    bt::bwd_rows<bt::kDQ><<<grid, L::kThreads, L::kSmemBytes, st>>>(q128, o128, k64, v64, mb, ra);
+    CUDA_TRY(cudaGetLastError());
+  }
+  {
+    using L = bt::RowsLayout<bt::kDKDV>;
+    ra.out1 = dK;
+    ra.out2 = dV;
+    const dim3 grid(mtiles, (rows + L::kR - 1) / L::kR, tri::kHeads);
+    bt::bwd_rows<bt::kDKDV><<<grid, L::kThreads, L::kSmemBytes, st>>>(k128, v128, q64, o64, mbT,
+                                                                       ra);
+    CUDA_TRY(cudaGetLastError());
+  }
+  {
+    bt::DbiasArgs da{};
+    da.nlse2 = w.nlse2;
+    da.nD = w.nD;
+    da.dB = dbias;
+    da.N = N;
+    da.rows = rows;
+    da.ld = ld;
+    da.status = w.status;
+    const dim3 grid((N + bt::kTN - 1) / bt::kTN, mtiles, tri::kHeads);
+    bt::bwd_dbias_tc<<<grid, bt::kDbThreads, bt::kDbSmemBytes, st>>>(q128, o128, k64, v64, mb, da);
+    CUDA_TRY(cudaGetLastError());
+  }
+  return core_finish(w, st, flags);
 }

@@ -49,7 +49,8 @@
 // rescaled in TMEM (then only after the previous PV has completed, which the
 // commit of the QK issued right after it signals); p = 2^(s - m) is at most 2^kTau.  The offset starts
 // at a finite floor so fully-masked tiles (bias -3e38) give p = 0, never NaN;
-// a row whose keys are all masked ends with l = 0 and writes o = 0.
+// a row whose keys are all masked ends with l = 0 and writes o = 0 (and, when
+// asked for, lse = +inf).
 //
 // Every mbarrier wait is bounded (sm100.cuh); on expiry the CTA records
 // TRI_ATTN_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
@@ -404,6 +405,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        // the row's natural-log log-sum-exp, ln 2 * (m + log2 l), for a backward pass
+        if (a.lse != nullptr)
+          a.lse[(static_cast<long long>(row) * kHeads + h) * a.N + j] =
+              l_sum > 0.f ? (m_used + __log2f(l_sum)) * 0.69314718055994531f : INFINITY;
       }
     } else if (lane == 0) {
       *abort_flag = 1;

@@ -169,3 +169,42 @@ def test_core_forward_rejects_bad_arguments_without_device():
     assert call(rows=70000) == binding.TRI_ATTN_ERR_UNSUPPORTED
     if not torch.cuda.is_available():
         assert call() == binding.TRI_ATTN_ERR_NO_DEVICE
+
+
+def test_tensor_core_core_calls_reject_bad_arguments_without_device():
+    L = binding.lib()
+    ws_bytes = binding.tri_attn_attention_bf16_workspace_bytes
+    assert ws_bytes(0, 10) == 0 and ws_bytes(3, 0) == 0
+    # status word, Qs, b2 and b2T, -lse2 and -D, each 256-byte aligned (ld = 128 here)
+    al = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    want = al(4) + al(3 * 4 * 70 * 32 * 2) + 2 * al(4 * 70 * 128 * 2) + 2 * al(3 * 4 * 128 * 4)
+    assert ws_bytes(3, 70) == want
+    buf = 0x10000
+    fwd = dict(Q=buf, K=buf, V=buf, bias=buf, mask=None, rows=3, N=70, O=buf, lse=buf,
+               workspace=buf, workspace_bytes=want, stream=None, flags=0)
+    bwd = dict(Q=buf, K=buf, V=buf, bias=buf, mask=None, O=buf, lse=buf, dO=buf, rows=3, N=70,
+               dQ=buf, dK=buf, dV=buf, dbias=buf, workspace=buf, workspace_bytes=want,
+               stream=None, flags=0)
+
+    def f(**kw):
+        return L.tri_attn_attention_forward_bf16(*dict(fwd, **kw).values())
+
+    def b(**kw):
+        return L.tri_attn_attention_backward_bf16(*dict(bwd, **kw).values())
+
+    bad = binding.TRI_ATTN_ERR_INVALID_ARG
+    for call in (f, b):
+        assert call(Q=None) == bad
+        assert call(V=buf + 8) == bad  # misaligned
+        assert call(bias=None) == bad
+        assert call(rows=0) == bad and call(N=0) == bad
+        assert call(workspace=None) == bad
+        assert call(workspace_bytes=want - 1) == bad
+        assert call(rows=70000, workspace_bytes=ws_bytes(70000, 70)) == \
+            binding.TRI_ATTN_ERR_UNSUPPORTED
+        assert call(lse=buf + 2) == bad
+    assert b(lse=None) == bad and b(dO=None) == bad and b(dbias=buf + 4) == bad
+    if not torch.cuda.is_available():
+        assert f() == binding.TRI_ATTN_ERR_NO_DEVICE
+        assert f(lse=None) == binding.TRI_ATTN_ERR_NO_DEVICE  # lse is optional in the forward
+        assert b() == binding.TRI_ATTN_ERR_NO_DEVICE

@@ -1,0 +1,155 @@
+"""Parity of the tensor-core attention core with the fp64 oracle.
+
+tri_attn_attention_forward_bf16 and tri_attn_attention_backward_bf16 take
+bf16 operands and accumulate in fp32.  The oracle runs on the same
+bf16-rounded inputs.  Checks:
+- element by element, at sizes that span several tiles and a ragged tail, with
+  masks, with row counts that leave the kernels' row groups partly empty, on an
+  all-masked problem and at N = 1;
+- at N = 768 (every row on the GPU): sampled rows of dQ, dK and dV, and
+  sampled query lines of the bias gradient, against the oracle;
+- the softmax-Jacobian property sum_k dbias[h][j][k] = 0;
+- bitwise determinism."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from protein_pair_representation_layernorm_b200 import binding
+from gpu_util import PARITY_LOG
+
+pytestmark = pytest.mark.gpu
+
+H, D = 4, 32
+# Tolerances, from the arithmetic: q * log2(e)/sqrt(d) and the base-2 bias are
+# rounded to bf16 before the score MMA, and P and ds to bf16 before the
+# gradient MMAs (relative 2^-9 each); on these O(1) logits that moves a
+# probability by a few tenths of a percent, and every sum runs in fp32.
+GRAD_REL_L2 = 1e-2
+GRAD_MAX_REL = 4e-2  # max |error| relative to the largest |gradient|
+O_REL_L2, O_MAX_ABS = 5e-3, 2e-2  # the bf16 tolerance of the attention output
+P_MAX_ABS = 1e-2  # probabilities implied by the returned lse, against the oracle's
+
+
+def _inputs(seed, rows, N, mask_kind):
+    rng = np.random.default_rng(seed)
+    bf = lambda a: torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16)  # noqa: E731
+    q, k, v, g = (bf(rng.normal(size=(rows, H, N, D))) for _ in range(4))
+    bias = bf(rng.normal(size=(H, N, N)))
+    if mask_kind is None:
+        mask = None
+    elif mask_kind == "random":
+        mask = (rng.random(N) > 0.2).astype(np.uint8)
+    elif mask_kind == "head":
+        mask = np.ones(N, np.uint8)
+        mask[:10] = 0
+    elif mask_kind == "all":
+        mask = np.zeros(N, np.uint8)
+    return q, k, v, g, bias, mask
+
+
+def _gpu(q, k, v, g, bias, mask):
+    m = None if mask is None else torch.from_numpy(mask).cuda()
+    Q, K, V, G, B = (t.cuda() for t in (q, k, v, g, bias))
+    O, lse = binding.attention_forward_bf16(Q, K, V, B, m)
+    grads = binding.attention_backward_bf16(Q, K, V, B, O, lse, G, m, sync=True)
+    torch.cuda.synchronize()
+    return O.float().cpu().numpy(), lse.cpu().numpy(), [t.cpu().numpy().astype(np.float64)
+                                                        for t in grads]
+
+
+def _f64(t):
+    return t.float().numpy().astype(np.float64)
+
+
+def _to_oracle(a):  # [rows][H][N][d] -> (rows, N, H, d)
+    return np.ascontiguousarray(a.transpose(0, 2, 1, 3))
+
+
+def _check(name, got, ref):
+    scale = max(float(np.abs(ref).max()), 1e-30)
+    err = float(np.abs(got - ref).max())
+    rel_l2 = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
+    PARITY_LOG.append(f"tensor-core backward {name}: rel_l2 {rel_l2:.2e}, "
+                      f"max_abs/max {err / scale:.2e}")
+    assert rel_l2 <= GRAD_REL_L2 and err <= GRAD_MAX_REL * scale + 1e-6, (name, rel_l2, err, scale)
+
+
+def _check_forward(tag, q, k, v, bias, mask, O, lse):
+    """o against the oracle's attention; lse through the probabilities it implies."""
+    qo, ko, vo = (_to_oracle(_f64(t)) for t in (q, k, v))
+    b = _f64(bias)
+    rows, N = qo.shape[0], qo.shape[1]
+    for r in range(rows):
+        o_ref, p_ref = oracle.attend(qo[r], ko[r], vo[r], b, mask, want_probs=True)
+        o_got = _to_oracle(O)[r]
+        rel = float(np.linalg.norm(o_got - o_ref) / max(np.linalg.norm(o_ref), 1e-30))
+        mx = float(np.abs(o_got - o_ref).max())
+        assert rel <= O_REL_L2 and mx <= O_MAX_ABS, (tag, r, rel, mx)
+        # s_jk in natural units from the same bf16 inputs; p = exp(s - lse)
+        s = np.einsum("jhd,khd->hjk", qo[r], ko[r]) / np.sqrt(D) + b
+        with np.errstate(invalid="ignore", over="ignore"):
+            p_got = np.exp(s - lse[r][:, :, None])
+        if mask is not None:
+            p_got[:, :, mask == 0] = 0.0
+        p_got[~np.isfinite(p_got)] = 0.0
+        assert float(np.abs(p_got - p_ref).max()) <= P_MAX_ABS, (tag, r)
+
+
+@pytest.mark.parametrize("rows,N,mask_kind,seed", [
+    (4, 70, None, 11), (5, 133, "random", 12), (2, 64, "head", 13), (3, 200, "random", 14),
+    (1, 1, None, 15), (2, 257, None, 16)])
+def test_tensor_core_core_matches_oracle(rows, N, mask_kind, seed):
+    q, k, v, g, bias, mask = _inputs(seed, rows, N, mask_kind)
+    O, lse, (dq, dk, dv, db) = _gpu(q, k, v, g, bias, mask)
+    tag = f"N={N} rows={rows} mask={mask_kind}"
+    _check_forward(tag, q, k, v, bias, mask, O, lse)
+    rq, rk, rv, rb = oracle.tri_attn_core_bwd(*(_to_oracle(_f64(t)) for t in (q, k, v)),
+                                              _f64(bias), _to_oracle(_f64(g)), mask)
+    _check(f"dQ {tag}", _to_oracle(dq), rq)
+    _check(f"dK {tag}", _to_oracle(dk), rk)
+    _check(f"dV {tag}", _to_oracle(dv), rv)
+    _check(f"dbias {tag}", db, rb)
+
+
+def test_tensor_core_all_masked():
+    """Every key masked: o = 0, lse = +inf, every gradient exactly 0."""
+    q, k, v, g, bias, mask = _inputs(17, 2, 40, "all")
+    O, lse, grads = _gpu(q, k, v, g, bias, mask)
+    assert not np.any(O)
+    assert np.all(np.isposinf(lse))
+    for t in grads:
+        assert not np.any(t)
+
+
+def test_tensor_core_backward_is_deterministic():
+    q, k, v, g, bias, mask = _inputs(18, 3, 150, "random")
+    a = _gpu(q, k, v, g, bias, mask)
+    b = _gpu(q, k, v, g, bias, mask)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    for x, y in zip(a[2], b[2]):
+        assert np.array_equal(x, y)
+
+
+def test_tensor_core_full_size_sampled():
+    """N = 768 with every row: rows 0, 383 and 767 of dQ, dK, dV and query
+    lines 0, 400 and 767 of the bias gradient (summed over all 768 rows)
+    against the oracle; sum_k dbias[h][j][k] = 0 for every (h, j)."""
+    N, rows = 768, 768
+    q, k, v, g, bias, mask = _inputs(19, rows, N, "random")
+    _, _, (dq, dk, dv, db) = _gpu(q, k, v, g, bias, mask)
+    qo, ko, vo, go = (_to_oracle(_f64(t)) for t in (q, k, v, g))
+    b = _f64(bias)
+    for r in (0, 383, 767):
+        rq, rk, rv, _ = oracle.attend_bwd(qo[r], ko[r], vo[r], b, go[r], mask)
+        _check(f"dQ N=768 row {r}", _to_oracle(dq)[r], rq)
+        _check(f"dK N=768 row {r}", _to_oracle(dk)[r], rk)
+        _check(f"dV N=768 row {r}", _to_oracle(dv)[r], rv)
+    for j in (0, 400, 767):
+        ref = np.zeros((H, N))
+        for r in range(rows):
+            ref += oracle.attend_bwd(qo[r][j:j + 1], ko[r], vo[r], b[:, j:j + 1, :],
+                                     go[r][j:j + 1], mask)[3][:, 0, :]
+        _check(f"dbias N=768 line {j}", db[:, j, :], ref)
+    row_sums = np.abs(db.sum(axis=2)).max()
+    assert row_sums <= 1e-3 * np.abs(db).sum(axis=2).max(), row_sums
