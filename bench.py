@@ -51,11 +51,11 @@ NUM_SMS = 148
 SM_MAX_MHZ = 1965.0
 
 # DRAM bytes per tri_attn_fwd launch at N = 1536, from one ncu capture of this
-# kernel source at N = 768 (ending node; 457.8 MB read + 133.9 MB written)
+# kernel source at N = 768 (457.8 MB read + 133.4 MB written)
 # scaled by the ratio of pairs (4): Q, K, V read once, O written once, and the
 # logit bias all grow with N^2.  Valid only for the source with this hash;
 # otherwise reported as null.
-TRAFFIC = {"tri_attn_fwd.cuh": "d277a929470fd6db", "bytes_per_launch": 4 * (457.800192e6 + 133.886464e6),
+TRAFFIC = {"tri_attn_fwd.cuh": "1c1f0e05cae114b9", "bytes_per_launch": 4 * (457.754880e6 + 133.433344e6),
            "measured_at": "N=768, scaled x4 to N=1536"}
 
 
@@ -70,7 +70,9 @@ def parse():
                     help="workload index (the metric is quoted on the default; others are for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward", action="store_true",
-                    help="time the attention-core backward (fp32) instead; one JSON line")
+                    help="time the attention-core backward (bf16, tensor cores) instead; one JSON line")
+    ap.add_argument("--backward-f32", action="store_true",
+                    help="with --backward: the fp32 SIMT kernels instead of the tensor-core ones")
     return ap.parse_args()
 
 
@@ -411,10 +413,13 @@ def run_ours(args, world, rank, local):
 
 
 def run_backward(args, rank):
-    """Time tri_attn_attention_backward (fp32 SIMT kernels) on the workload's N
-    with every row, on synthetic q, k, v, dO and bias; prints one JSON line.
-    Algorithmic work: 10 d flop per (row, head, query, unmasked key) score
-    (S and dP, 2 d each, recomputed once; dQ, dK and dV, 2 d each)."""
+    """Time the attention-core backward on the workload's N with every row, on
+    synthetic q, k, v, dO and bias; prints one JSON line.  Default: the
+    tensor-core path (tri_attn_attention_backward_bf16, after one
+    tri_attn_attention_forward_bf16 for o and lse); --backward-f32: the fp32
+    SIMT kernels (tri_attn_attention_backward).  Algorithmic work: 10 d flop
+    per (row, head, query, unmasked key) score (S and dP, 2 d each, once;
+    dQ, dK and dV, 2 d each)."""
     if rank != 0:
         return
     import ctypes
@@ -425,22 +430,46 @@ def run_backward(args, rank):
     N = inp.N
     rows = N
     H, d = 4, 32
+    tc = not args.backward_f32
+    dt = torch.bfloat16 if tc else torch.float32
     gen = torch.Generator(device="cuda").manual_seed(17)
-    Q, K, V, dO = (torch.randn(rows, H, N, d, device="cuda", generator=gen) for _ in range(4))
-    bias = torch.randn(H, N, N, device="cuda", generator=gen)
+    Q, K, V, dO = (torch.randn(rows, H, N, d, device="cuda", generator=gen).to(dt)
+                   for _ in range(4))
+    bias = torch.randn(H, N, N, device="cuda", generator=gen).to(dt)
     mask = None if inp.mask is None else inp.mask.cuda().to(torch.uint8).contiguous()
     n_valid = N if inp.mask is None else int(inp.mask.sum())
-    dQ, dK, dV, dB = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(bias)
-    nbytes = binding.tri_attn_attention_backward_workspace_bytes(rows, N)
-    ws = torch.empty(nbytes // 4, dtype=torch.float32, device="cuda")
+    f32 = dict(dtype=torch.float32, device="cuda")
+    dQ, dK, dV = (torch.empty(rows, H, N, d, **f32) for _ in range(3))
+    dB = torch.empty(H, N, N, **f32)
     st = torch.cuda.Stream()
     P = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())  # noqa: E731
-
-    def step():
-        rc = binding.tri_attn_attention_backward(P(Q), P(K), P(V), P(bias), P(mask), P(dO), rows, N,
-                                                 P(dQ), P(dK), P(dV), P(dB), P(ws), nbytes,
-                                                 ctypes.c_void_p(st.cuda_stream), 0)
+    sp = ctypes.c_void_p(st.cuda_stream)
+    if tc:
+        nbytes = binding.tri_attn_attention_bf16_workspace_bytes(rows, N)
+        ws = torch.empty((nbytes + 15) // 16 * 4, **f32)
+        O = torch.empty_like(Q)
+        lse = torch.empty(rows, H, N, **f32)
+        rc = binding.tri_attn_attention_forward_bf16(P(Q), P(K), P(V), P(bias), P(mask), rows, N,
+                                                     P(O), P(lse), P(ws), nbytes, sp,
+                                                     binding.TRI_ATTN_FLAG_SYNC)
         assert rc == binding.TRI_ATTN_OK, binding.tri_attn_status_string(rc)
+
+        def step():
+            rc = binding.tri_attn_attention_backward_bf16(
+                P(Q), P(K), P(V), P(bias), P(mask), P(O), P(lse), P(dO), rows, N, P(dQ), P(dK),
+                P(dV), P(dB), P(ws), nbytes, sp, 0)
+            assert rc == binding.TRI_ATTN_OK, binding.tri_attn_status_string(rc)
+        launches = 6  # prep_q, prep_bias, prep_rows, dQ, dK dV, dbias
+    else:
+        nbytes = binding.tri_attn_attention_backward_workspace_bytes(rows, N)
+        ws = torch.empty(nbytes // 4, **f32)
+
+        def step():
+            rc = binding.tri_attn_attention_backward(P(Q), P(K), P(V), P(bias), P(mask), P(dO),
+                                                     rows, N, P(dQ), P(dK), P(dV), P(dB), P(ws),
+                                                     nbytes, sp, 0)
+            assert rc == binding.TRI_ATTN_OK, binding.tri_attn_status_string(rc)
+        launches = 4
 
     for _ in range(max(args.warmup, 1)):
         step()
@@ -454,17 +483,24 @@ def run_backward(args, rank):
     ms = ev0.elapsed_time(ev1) / args.steps
     flops = 10.0 * d * rows * N * n_valid * H
     tf = flops / (ms / 1e3) / 1e12
-    # fp32 FFMA peak: 148 SMs x 128 lanes x 2 flop x 1965 MHz
-    peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    if tc:
+        peak_tf, _, peak_src = measured_peaks()
+        roof = {"bound": "tensor", "achieved": tf, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": tf / peak_tf, "peak_source": f"{peak_src} bf16_tflops (burst)"}
+    else:
+        # fp32 FFMA peak: 148 SMs x 128 lanes x 2 flop x 1965 MHz
+        peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        roof = {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                "frac": tf / peak,
+                "peak_derivation": "fp32 FFMA: 148 SMs x 128 lanes x 2 flop x 1965 MHz"}
     print(json.dumps({
         "metric": "attention-core backward TFLOP/s (algorithmic: 10 d flop per unmasked score)",
         "value": tf, "unit": "TFLOP/s", "ms_per_step": ms, "steps": args.steps,
-        "warmup": max(args.warmup, 1), "higher_is_better": True, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": w.name, "N": N, "rows": rows, "heads": H, "head_dim": d},
-        "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
-                     "frac": tf / peak,
-                     "peak_derivation": "fp32 FFMA: 148 SMs x 128 lanes x 2 flop x 1965 MHz"},
-        "gpu_launches": 4 * args.steps}), flush=True)
+        "warmup": max(args.warmup, 1), "higher_is_better": True,
+        "dtype": "bf16" if tc else "f32", "data": "synthetic",
+        "config": {"workload": w.name, "N": N, "rows": rows, "heads": H, "head_dim": d,
+                   "path": "tensor cores (tcgen05)" if tc else "fp32 SIMT"},
+        "roofline": roof, "gpu_launches": launches * args.steps}), flush=True)
 
 
 def main():

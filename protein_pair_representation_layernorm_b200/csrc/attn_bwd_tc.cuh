@@ -14,10 +14,14 @@
 // grandes").  Three tensor-core kernels recompute the scores and dP = dO V^T of
 // their tiles from the forward's row statistics instead of storing p (an
 // R x N x N x H tensor):
-//   bwd_rows<kDQ>    CTA = 3 rows x 128 queries x head; walks the keys in tiles
+//   bwd_rows<kDQ>    CTA = 2 rows x 128 queries x head; walks the keys in tiles
 //                    of 64: S = Qs K^T and dP = dO V^T (SS MMAs into TMEM), ds in
 //                    the softmax threads (thread = query = TMEM lane), written
-//                    back to TMEM as bf16, then dQ += ds K (TS MMA).
+//                    back to TMEM as bf16, then dQ += ds K (TS MMA).  ds has
+//                    TMEM columns of its own, so the scores of step t+1 are
+//                    computed as soon as the threads hold those of step t in
+//                    registers, and the gradient MMAs of step t run while they
+//                    work on step t+1.
 //   bwd_rows<kDKDV>  CTA = 2 rows x 128 keys x head; the same walk over the
 //                    queries with the roles of queries and keys exchanged:
 //                    S^T = K Qs^T, dP^T = V dO^T, thread = key, then
@@ -150,13 +154,17 @@ struct RowsArgs {
 // (kDKDV).  A stage per step of 64 columns: the bias tile shared by the rows
 // (128 x 64 bf16, 128-byte swizzle) and per row X1, X2 (64 x 32): K and V
 // (kDQ), Qs and dO (kDKDV), plus for kDKDV the step's -lse2 and -D (64 fp32
-// each).  TMEM per row: S at +0 (P as bf16 over its first 32 columns, kDKDV),
-// dP at +64 (ds as bf16 over its first 32 columns), the accumulators at +128
-// (dQ; or dK, then dV at +160).
+// each).  TMEM per row: S at +0, dP at +64, then ds (bf16, 32 columns) at
+// +128, P (bf16, kDKDV) at +160, and the accumulators: dQ at +160 (kDQ), or
+// dK at +192 and dV at +224 (kDKDV).  ds and P have columns of their own, so
+// the scores of step t+1 are computed while the warps still work on step t.
 template <int kMode>
 struct RowsLayout {
-  static constexpr int kR = kMode == kDQ ? 3 : 2;
-  static constexpr int kRowCols = kMode == kDQ ? 160 : 192;
+  static constexpr int kR = 2;
+  static constexpr int kRowCols = kMode == kDQ ? 192 : 256;
+  static constexpr int kColDS = 128;
+  static constexpr int kColP = 160;
+  static constexpr int kColAcc = kMode == kDQ ? 160 : 192;
   static constexpr int kStages = 4;
   static constexpr int kProducerWarp = 4 * kR;
   static constexpr int kMmaWarp0 = 4 * kR + 1;  // MMA warp of row g: kMmaWarp0 + g
@@ -175,8 +183,9 @@ struct RowsLayout {
   static constexpr uint32_t kStageTx = kStVec + 2 * kR * kVecBytes;
   static constexpr uint32_t kStageBytes = (kStageTx + 1023) / 1024 * 1024;
   static constexpr uint32_t kSmemBar = kSmemStages + kStages * kStageBytes;
-  // a_full, st_full[S], st_empty[S], s_full[R], ds_full[R], acc_full[R], drain[R]
-  static constexpr uint32_t kNumBars = 1 + 2 * kStages + 4 * kR;
+  // a_full, st_full[S], st_empty[S], s_full[R], s_read[R], ds_full[R], acc_done[R],
+  // acc_full[R], drain[R]
+  static constexpr uint32_t kNumBars = 1 + 2 * kStages + 6 * kR;
   static constexpr uint32_t kSmemBytes = kSmemBar + kNumBars * 8 + 16 + 1024;
   static_assert(kSmemStages % 1024 == 0 && kStageBytes % 1024 == 0 && kStX1 % 1024 == 0,
                 "swizzled tiles need 1024-byte alignment");
@@ -199,8 +208,10 @@ __global__ void __launch_bounds__(RowsLayout<kMode>::kThreads, 1)
   uint64_t* st_full = a_full + 1;
   uint64_t* st_empty = st_full + kStages;  // one commit per row's MMA warp
   uint64_t* s_full = st_empty + kStages;   // [g]: S(t) and dP(t) of row g in TMEM
-  uint64_t* ds_full = s_full + kR;         // [g]: ds(t) (and P(t)) of row g in TMEM
-  uint64_t* acc_full = ds_full + kR;       // [g]: every MMA of row g complete
+  uint64_t* s_read = s_full + kR;          // [g]: the warps of row g hold S(t), dP(t) in registers
+  uint64_t* ds_full = s_read + kR;         // [g]: ds(t) (and P(t)) of row g in TMEM
+  uint64_t* acc_done = ds_full + kR;       // [g]: the gradient MMAs of step t have read ds(t), P(t)
+  uint64_t* acc_full = acc_done + kR;      // [g]: every MMA of row g complete
   uint64_t* drain = acc_full + kR;         // [g]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -219,7 +230,9 @@ __global__ void __launch_bounds__(RowsLayout<kMode>::kThreads, 1)
     }
     for (int g = 0; g < kR; ++g) {
       mbar_init(&s_full[g], 1);
+      mbar_init(&s_read[g], 4);
       mbar_init(&ds_full[g], 4);
+      mbar_init(&acc_done[g], 1);
       mbar_init(&acc_full[g], 1);
       mbar_init(&drain[g], 1);
     }
@@ -299,7 +312,8 @@ __global__ void __launch_bounds__(RowsLayout<kMode>::kThreads, 1)
       const uint64_t a_hi = dA & 0xFFFFFFFF00000000ull, st_hi = dSt & 0xFFFFFFFF00000000ull;
       auto adesc = [&](uint32_t off) { return a_hi | (a_lo + (off >> 4)); };
       auto sdesc = [&](uint32_t off) { return st_hi | (st_lo + (off >> 4)); };
-      const uint32_t tS = tmem + g * L::kRowCols, tDP = tS + 64, tAcc = tS + 128;
+      const uint32_t tS = tmem + g * L::kRowCols, tDP = tS + 64;
+      const uint32_t tDS = tS + L::kColDS, tP = tS + L::kColP, tAcc = tS + L::kColAcc;
       // S = A1 X1^T and dP = A2 X2^T of stage s (K = 32: two K = 16 steps each)
       auto issue_sdp = [&](int s) {
 #pragma unroll
@@ -320,39 +334,41 @@ __global__ void __launch_bounds__(RowsLayout<kMode>::kThreads, 1)
       auto issue_acc = [&](int s, bool first) {
 #pragma unroll
         for (int kc = 0; kc < kTN / 16; ++kc)
-          mma_ts(tAcc, tDP + kc * 8,
+          mma_ts(tAcc, tDS + kc * 8,
                  sdesc(s * L::kStageBytes + L::kStX1 + g * L::kXTile + kc * 1024), kIdTS,
                  (!first || kc > 0) ? 1u : 0u);
         if constexpr (kMode == kDKDV) {
 #pragma unroll
           for (int kc = 0; kc < kTN / 16; ++kc)
-            mma_ts(tAcc + 32, tS + kc * 8,
+            mma_ts(tAcc + 32, tP + kc * 8,
                    sdesc(s * L::kStageBytes + L::kStX2 + g * L::kXTile + kc * 1024), kIdTS,
                    (!first || kc > 0) ? 1u : 0u);
         }
+        mma_commit(&acc_done[g]);
         mma_commit(&st_empty[s]);  // this row's MMAs on stage s
       };
-      bool ok = mbar_wait(a_full, 0, abort_flag);
+      bool ok = mbar_wait(a_full, 0, abort_flag) && mbar_wait(&st_full[0], 0, abort_flag);
       bool issued = false;
-      for (int t = 0; ok && t < T; ++t) {
-        const int s = t % kStages;
-        if (!(ok = mbar_wait(&st_full[s], (t / kStages) & 1, abort_flag))) break;
-        if (t > 0) {
-          // ds(t-1) is in TMEM: accumulate it, then overwrite S and dP (the
-          // tensor core runs one thread's MMAs in order)
-          if (!(ok = mbar_wait(&ds_full[g], (t - 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          issue_acc((t - 1) % kStages, t == 1);
-        }
+      if (ok) {
         tc_fence_after();
-        issue_sdp(s);
+        issue_sdp(0);
         issued = true;
       }
-      if (ok && (ok = mbar_wait(&ds_full[g], (T - 1) & 1, abort_flag))) {
+      for (int t = 0; ok && t < T; ++t) {
+        if (t + 1 < T) {
+          // S(t+1), dP(t+1) as soon as the warps hold S(t), dP(t) in registers
+          const int s1 = (t + 1) % kStages;
+          if (!(ok = mbar_wait(&st_full[s1], ((t + 1) / kStages) & 1, abort_flag))) break;
+          if (!(ok = mbar_wait(&s_read[g], t & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_sdp(s1);
+        }
+        // the gradient products of step t once ds(t) (and P(t)) are in TMEM
+        if (!(ok = mbar_wait(&ds_full[g], t & 1, abort_flag))) break;
         tc_fence_after();
-        issue_acc((T - 1) % kStages, T == 1);
-        mma_commit(&acc_full[g]);
+        issue_acc(t % kStages, t == 0);
       }
+      if (ok) mma_commit(&acc_full[g]);
       if (!ok) {
         *abort_flag = 1;
         report_status(a.status, kStatusTimeout);
@@ -411,6 +427,14 @@ __global__ void __launch_bounds__(RowsLayout<kMode>::kThreads, 1)
           bw[4 * c + 3] = v.w;
         }
         tmem_ld_wait();
+        tmem_regs_ready(sr);
+        tmem_regs_ready(dr);
+        if (half == 1) {
+          // S(t) and dP(t) are in registers: the MMAs of step t+1 may overwrite them
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_read[g]);
+        }
         uint32_t pds[16], pp[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -434,11 +458,18 @@ __global__ void __launch_bounds__(RowsLayout<kMode>::kThreads, 1)
           pds[e] = pack_bf16x2(ds.x, ds.y);
           if constexpr (kMode == kDKDV) pp[e] = pack_bf16x2(p.x, p.y);
         }
-        // ds over the dP columns already read (half 0 writes columns 0-15 of dP,
-        // half 1 columns 16-31, both read in half 0); P likewise over S
-        tmem_st16(tS + 64 + 16 * half, pds);
-        if constexpr (kMode == kDKDV) tmem_st16(tS + 16 * half, pp);
+        if (half == 0 && t > 0) {
+          // ds and P of step t-1 must have been read by its gradient MMAs
+          if (!__all_sync(0xffffffffu, mbar_wait(&acc_done[g], (t - 1) & 1, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        tmem_st16(tS + L::kColDS + 16 * half, pds);
+        if constexpr (kMode == kDKDV) tmem_st16(tS + L::kColP + 16 * half, pp);
       }
+      if (!ok) break;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -451,8 +482,9 @@ __global__ void __launch_bounds__(RowsLayout<kMode>::kThreads, 1)
       const bool live = row < a.rows && m < a.N;
       const long long orow = ((static_cast<long long>(row) * kHeads + h) * a.N + m) * kD;
       uint32_t v[32];
-      tmem_ld32(tS + 128, v);
+      tmem_ld32(tS + L::kColAcc, v);
       tmem_ld_wait();
+      tmem_regs_ready(v);
       // dQ = (ds K) / sqrt(d);  dK = (ds^T Qs) / (log2(e)/sqrt(d) * sqrt(d)) = ln 2 (ds^T Qs)
       const float sc = kMode == kDQ ? kInvSqrtD : kLn2;
       if (live) {
@@ -463,8 +495,9 @@ __global__ void __launch_bounds__(RowsLayout<kMode>::kThreads, 1)
                                __uint_as_float(v[4 * q + 2]) * sc, __uint_as_float(v[4 * q + 3]) * sc);
       }
       if constexpr (kMode == kDKDV) {
-        tmem_ld32(tS + 160, v);
+        tmem_ld32(tS + L::kColAcc + 32, v);
         tmem_ld_wait();
+        tmem_regs_ready(v);
         if (live) {
           float4* dst = reinterpret_cast<float4*>(a.out2 + orow);
 #pragma unroll
@@ -680,6 +713,8 @@ __global__ void __launch_bounds__(kDbThreads, 2)
           bw[4 * c + 3] = v.w;
         }
         tmem_ld_wait();
+        tmem_regs_ready(sr);
+        tmem_regs_ready(dr);
         if (half == 1) {
           // both halves of this buffer are in registers: the MMAs of row r+2 may overwrite it
           tc_fence_before();

@@ -313,6 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                  ((qc ^ sw64) << 4));
       }
       tmem_ld_wait();
+      tmem_regs_ready(v);
       uint32_t pk[8];
 #pragma unroll
       for (int q2 = 0; q2 < 2; ++q2) {
@@ -347,6 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(t_d + lane_base + 64 * hc + 32 * cc, v);
       tmem_ld16(t_z + lane_base + 32 * hc + 16 * cc, zv);
       tmem_ld_wait();
+      tmem_regs_ready(v);
+      tmem_regs_ready(zv);
 #pragma unroll
       for (int qq = 0; qq < 4; ++qq) {
         const int c = 4 * cc + qq, ch = 64 * hc + 8 * c;

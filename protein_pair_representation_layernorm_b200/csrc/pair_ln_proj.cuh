@@ -353,6 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t v[32];
           tmem_ld32(col0 + cc * 32, v);
           tmem_ld_wait();
+          tmem_regs_ready(v);
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             pk[cc][e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);

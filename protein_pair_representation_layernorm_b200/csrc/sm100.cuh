@@ -267,6 +267,19 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// tcgen05.ld fills its registers asynchronously: they hold the loaded values
+// only once tcgen05.wait::ld has completed, which the compiler does not know.
+// Arithmetic on them touches no memory, so the memory clobber of the wait does
+// not keep it behind the wait either.  Passing every loaded register through
+// this empty statement after the wait redefines it there (the statement is
+// volatile, so it stays after the wait), and every use reads the redefined
+// value.  Call it right after tmem_ld_wait() for each array the loads filled.
+template <int N>
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
                    taddr),

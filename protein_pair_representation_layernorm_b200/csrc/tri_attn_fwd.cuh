@@ -321,6 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           bw[4 * c + 3] = v.w;
         }
         tmem_ld_wait();
+        tmem_regs_ready(sr);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           // s + b with the bf16 bias as the operand of a mixed-precision add (no
@@ -356,6 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t ov[32];
         tmem_ld32(colO, ov);
         tmem_ld_wait();
+        tmem_regs_ready(ov);
 #pragma unroll
         for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * scale);
         tmem_st32(colO, ov);
@@ -394,6 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ov[32];
       tmem_ld32(colO, ov);
       tmem_ld_wait();
+      tmem_regs_ready(ov);
       if (row < a.rows && j < a.N) {
         const float inv = l_sum > 0.f ? 1.0f / l_sum : 0.f;
         uint32_t pk[16];

@@ -153,3 +153,28 @@ def test_tensor_core_full_size_sampled():
         _check(f"dbias N=768 line {j}", db[:, j, :], ref)
     row_sums = np.abs(db.sum(axis=2)).max()
     assert row_sums <= 1e-3 * np.abs(db).sum(axis=2).max(), row_sums
+
+
+def test_autograd_op_on_bf16_inputs():
+    """binding.AttentionCore on bf16 tensors runs the tensor-core forward and
+    backward: its output equals attention_forward_bf16's, its gradients
+    (returned in bf16) the fp32 gradients of attention_backward_bf16 rounded,
+    and both agree with the oracle."""
+    q, k, v, g, bias, mask = _inputs(20, 3, 90, "random")
+    m = torch.from_numpy(mask).cuda()
+    leaves = [t.cuda().requires_grad_() for t in (q, k, v, bias)]
+    out = binding.AttentionCore.apply(*leaves, m)
+    out.backward(g.cuda())
+    Q, K, V, B = (t.detach() for t in leaves)
+    O, lse = binding.attention_forward_bf16(Q, K, V, B, m)
+    assert torch.equal(out.detach(), O)
+    want = binding.attention_backward_bf16(Q, K, V, B, O, lse, g.cuda(), m, sync=True)
+    for leaf, w in zip(leaves, want):
+        assert leaf.grad.dtype == torch.bfloat16
+        assert torch.equal(leaf.grad, w.to(torch.bfloat16))
+    rq, rk, rv, rb = oracle.tri_attn_core_bwd(*(_to_oracle(_f64(t)) for t in (q, k, v)),
+                                              _f64(bias), _to_oracle(_f64(g)), mask)
+    for name, leaf, ref, tr in (("dQ", leaves[0], rq, True), ("dK", leaves[1], rk, True),
+                                ("dV", leaves[2], rv, True), ("dbias", leaves[3], rb, False)):
+        got = leaf.grad.float().cpu().numpy().astype(np.float64)
+        _check(f"autograd {name}", _to_oracle(got) if tr else got, ref)
