@@ -55,7 +55,7 @@ SM_MAX_MHZ = 1965.0
 # scaled by the ratio of pairs (4): Q, K, V read once, O written once, and the
 # logit bias all grow with N^2.  Valid only for the source with this hash;
 # otherwise reported as null.
-TRAFFIC = {"tri_attn_fwd.cuh": "1c1f0e05cae114b9", "bytes_per_launch": 4 * (457.754880e6 + 133.433344e6),
+TRAFFIC = {"tri_attn_fwd.cuh": "cb382a5e25ef7893", "bytes_per_launch": 4 * (457.797888e6 + 133.481472e6),
            "measured_at": "N=768, scaled x4 to N=1536"}
 
 
