@@ -68,7 +68,10 @@ extern "C" {
  * (2 s) expire, those threads free what they hold and leave, and the call
  * reports TRI_ATTN_ERR_TIMEOUT through the device status; the handle and the
  * CUDA context stay usable. */
-#define TRI_ATTN_FLAG_DEBUG_STALL   4u  /* tri_attn_fwd: one CTA's producer withholds its first stage */
+#define TRI_ATTN_FLAG_DEBUG_STALL   4u  /* tri_attn_fwd: one CTA's producer withholds its first stage
+                                       (also through tri_attn_attention_forward_bf16); in
+                                       tri_attn_attention_backward_bf16 the same in each of its
+                                       three tensor-core kernels */
 #define TRI_ATTN_FLAG_DEBUG_STALL_PROJ 8u   /* pair_ln_proj: one group of one CTA never gets its first
                                                tile of Z (every launch of the call) */
 #define TRI_ATTN_FLAG_DEBUG_STALL_GATE 16u  /* gate_out: one CTA's producer withholds its first stage
@@ -326,7 +329,7 @@ int tri_attn_attention_backward(const float *Q, const float *K, const float *V,
  * padded base-2 bias (and its transpose) and the per-query statistics.  Both
  * calls are asynchronous on `stream`; with TRI_ATTN_FLAG_SYNC they wait and
  * return the device status (TRI_ATTN_ERR_TIMEOUT if a kernel's bounded wait
- * expired).  The calls allocate nothing.
+ * expired; TRI_ATTN_FLAG_DEBUG_STALL injects that).  The calls allocate nothing.
  * Errors: TRI_ATTN_ERR_INVALID_ARG (NULL or misaligned pointer: Q, K, V, O,
  * dO, dQ, dK, dV, dbias and workspace must be 16-byte aligned, lse 4-byte;
  * rows or N < 1; workspace too small), TRI_ATTN_ERR_UNSUPPORTED (rows > 65535

@@ -146,6 +146,7 @@ struct RowsArgs {
   float* out1;         // dQ (kDQ) or dK (kDKDV): [rows][H][N][d]
   float* out2;         // dV (kDKDV)
   int N, rows, ld;
+  int debug_stall;     // fault injection: the producer of CTA 0 withholds its first stage
   int* status;
 };
 
@@ -262,6 +263,7 @@ __global__ void __launch_bounds__(RowsLayout<kMode>::kThreads, 1)
         tma_load_3d(smem + L::kSmemA1 + r * L::kATile, &map_a1, a_full, 0, m0, c2);
         tma_load_3d(smem + L::kSmemA2 + r * L::kATile, &map_a2, a_full, 0, m0, c2);
       }
+      const bool stall = a.debug_stall && blockIdx.x == 0 && rg == 0 && h == 0;
       int t_end = 0;
       for (int t = 0; t < T; ++t) {
         const int s = t % kStages;
@@ -271,6 +273,7 @@ __global__ void __launch_bounds__(RowsLayout<kMode>::kThreads, 1)
           break;
         }
         t_end = t + 1;
+        if (stall && t == 0) continue;  // fault injection: stage 0 is never filled
         uint8_t* st = smem + L::kSmemStages + s * L::kStageBytes;
         mbar_arrive_expect_tx(&st_full[s], L::kStageTx);
         tma_load_3d(st + L::kStB, &map_b, &st_full[s], t * kTN, m0, h);
@@ -294,7 +297,8 @@ __global__ void __launch_bounds__(RowsLayout<kMode>::kThreads, 1)
       if (!mbar_wait(a_full, 0, nullptr)) report_status(a.status, kStatusTimeout);
       for (int s = 0; s < kStages; ++s) {
         int last = -1;
-        for (int t = s; t < t_end; t += kStages) last = t;
+        for (int t = s; t < t_end; t += kStages)
+          if (!(stall && t == 0)) last = t;
         if (last >= 0 && !mbar_wait(&st_full[s], (last / kStages) & 1, nullptr))
           report_status(a.status, kStatusTimeout);
       }
@@ -526,6 +530,7 @@ struct DbiasArgs {
   const float* nD;     // [rows][H][ld]
   float* dB;           // [H][N][N]
   int N, rows, ld;
+  int debug_stall;     // fault injection: the producer of CTA 0 withholds its first stage
   int* status;
 };
 
@@ -606,6 +611,7 @@ __global__ void __launch_bounds__(kDbThreads, 2)
       tma_prefetch_desc(&map_b);
       mbar_arrive_expect_tx(b_full, kTM * kTN * 2);
       tma_load_3d(smem, &map_b, b_full, k0, j0, h);
+      const bool stall = a.debug_stall && blockIdx.x == 0 && blockIdx.y == 0 && h == 0;
       int r_end = 0;
       for (int r = 0; r < R; ++r) {
         const int s = r % kDbStages;
@@ -615,6 +621,7 @@ __global__ void __launch_bounds__(kDbThreads, 2)
           break;
         }
         r_end = r + 1;
+        if (stall && r == 0) continue;  // fault injection: stage 0 is never filled
         uint8_t* st = smem + kDbSmemStages + s * kDbStageBytes;
         const int c2 = r * kHeads + h;
         const long long voff = static_cast<long long>(c2) * a.ld + j0;
@@ -629,7 +636,8 @@ __global__ void __launch_bounds__(kDbThreads, 2)
       if (!mbar_wait(b_full, 0, nullptr)) report_status(a.status, kStatusTimeout);
       for (int s = 0; s < kDbStages; ++s) {
         int last = -1;
-        for (int r = s; r < r_end; r += kDbStages) last = r;
+        for (int r = s; r < r_end; r += kDbStages)
+          if (!(stall && r == 0)) last = r;
         if (last >= 0 && !mbar_wait(&st_full[s], (last / kDbStages) & 1, nullptr))
           report_status(a.status, kStatusTimeout);
       }

@@ -1491,6 +1491,7 @@ extern "C" int tri_attn_attention_forward_bf16(const void* Q, const void* K, con
   a.lse = lse;
   a.N = N;
   a.rows = rows;
+  a.debug_stall = (flags & TRI_ATTN_FLAG_DEBUG_STALL) ? 1 : 0;
   a.status = w.status;
   const dim3 grid((N + tri::attn::kBJ - 1) / tri::attn::kBJ,
                   (rows + tri::attn::kRows - 1) / tri::attn::kRows, tri::kHeads);
@@ -1543,6 +1544,7 @@ extern "C" int tri_attn_attention_backward_bf16(const void* Q, const void* K, co
   ra.N = N;
   ra.rows = rows;
   ra.ld = ld;
+  ra.debug_stall = (flags & TRI_ATTN_FLAG_DEBUG_STALL) ? 1 : 0;
   ra.status = w.status;
   const unsigned mtiles = static_cast<unsigned>((N + bt::kTM - 1) / bt::kTM);
   {
@@ -1570,6 +1572,7 @@ extern "C" int tri_attn_attention_backward_bf16(const void* Q, const void* K, co
     da.N = N;
     da.rows = rows;
     da.ld = ld;
+    da.debug_stall = (flags & TRI_ATTN_FLAG_DEBUG_STALL) ? 1 : 0;
     da.status = w.status;
     const dim3 grid((N + bt::kTN - 1) / bt::kTN, mtiles, tri::kHeads);
     bt::bwd_dbias_tc<<<grid, bt::kDbThreads, bt::kDbSmemBytes, st>>>(q128, o128, k64, v64, mb, da);

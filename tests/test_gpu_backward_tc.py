@@ -178,3 +178,44 @@ def test_autograd_op_on_bf16_inputs():
                                 ("dV", leaves[2], rv, True), ("dbias", leaves[3], rb, False)):
         got = leaf.grad.float().cpu().numpy().astype(np.float64)
         _check(f"autograd {name}", _to_oracle(got) if tr else got, ref)
+
+
+def test_withheld_copy_reports_timeout_and_recovers():
+    """A withheld stage in CTA 0 of each tensor-core kernel (forward: one; backward:
+    dQ, dK dV and dbias) makes its bounded waits expire: the call returns
+    TRI_ATTN_ERR_TIMEOUT with SYNC, the other CTAs finish, and the next call on the
+    same workspace and context is correct."""
+    import ctypes
+    q, k, v, g, bias, mask = _inputs(21, 2, 70, "random")
+    m = torch.from_numpy(mask).cuda()
+    Q, K, V, G, B = (t.cuda() for t in (q, k, v, g, bias))
+    rows, N = 2, 70
+    nbytes = binding.tri_attn_attention_bf16_workspace_bytes(rows, N)
+    ws = torch.empty((nbytes + 15) // 16 * 4, dtype=torch.float32, device="cuda")
+    O = torch.empty_like(Q)
+    lse = torch.empty(rows, H, N, dtype=torch.float32, device="cuda")
+    f32 = dict(dtype=torch.float32, device="cuda")
+    dq, dk, dv = (torch.empty(rows, H, N, D, **f32) for _ in range(3))
+    db = torch.empty(H, N, N, **f32)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    stall = binding.TRI_ATTN_FLAG_DEBUG_STALL | binding.TRI_ATTN_FLAG_SYNC
+    rc = binding.tri_attn_attention_forward_bf16(P(Q), P(K), P(V), P(B), P(m), rows, N, P(O),
+                                                 P(lse), P(ws), nbytes, None, stall)
+    assert rc == binding.TRI_ATTN_ERR_TIMEOUT, binding.tri_attn_status_string(rc)
+    rc = binding.tri_attn_attention_forward_bf16(P(Q), P(K), P(V), P(B), P(m), rows, N, P(O),
+                                                 P(lse), P(ws), nbytes, None,
+                                                 binding.TRI_ATTN_FLAG_SYNC)
+    assert rc == binding.TRI_ATTN_OK
+    args = (P(Q), P(K), P(V), P(B), P(m), P(O), P(lse), P(G), rows, N, P(dq), P(dk), P(dv), P(db),
+            P(ws), nbytes, None)
+    rc = binding.tri_attn_attention_backward_bf16(*args, stall)
+    assert rc == binding.TRI_ATTN_ERR_TIMEOUT, binding.tri_attn_status_string(rc)
+    rc = binding.tri_attn_attention_backward_bf16(*args, binding.TRI_ATTN_FLAG_SYNC)
+    assert rc == binding.TRI_ATTN_OK
+    got = [t.cpu().numpy().astype(np.float64) for t in (dq, dk, dv, db)]
+    rq, rk, rv, rb = oracle.tri_attn_core_bwd(*(_to_oracle(_f64(t)) for t in (q, k, v)),
+                                              _f64(bias), _to_oracle(_f64(g)), mask)
+    _check("dQ after timeout", _to_oracle(got[0]), rq)
+    _check("dK after timeout", _to_oracle(got[1]), rk)
+    _check("dV after timeout", _to_oracle(got[2]), rv)
+    _check("dbias after timeout", got[3], rb)
