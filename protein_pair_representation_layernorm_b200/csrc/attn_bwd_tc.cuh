@@ -14,19 +14,19 @@
 // grandes").  Three tensor-core kernels recompute the scores and dP = dO V^T of
 // their tiles from the forward's row statistics instead of storing p (an
 // R x N x N x H tensor):
-//   bwd_rows<kDQ>    CTA = 2 rows x 128 queries x head; walks the keys in tiles
+//   bwd_rows<kDQ>    CTA = 3 rows x 128 queries x head; walks the keys in tiles
 //                    of 64: S = Qs K^T and dP = dO V^T (SS MMAs into TMEM), ds in
 //                    the softmax threads (thread = query = TMEM lane), written
-//                    back to TMEM as bf16, then dQ += ds K (TS MMA).  ds has
-//                    TMEM columns of its own, so the scores of step t+1 are
-//                    computed as soon as the threads hold those of step t in
-//                    registers, and the gradient MMAs of step t run while they
-//                    work on step t+1.
+//                    back to TMEM as bf16, then dQ += ds K (TS MMA).
 //   bwd_rows<kDKDV>  CTA = 2 rows x 128 keys x head; the same walk over the
 //                    queries with the roles of queries and keys exchanged:
 //                    S^T = K Qs^T, dP^T = V dO^T, thread = key, then
 //                    dV += P^T dO and dK += ds^T Qs (two TS MMAs).  The per-query
-//                    statistics of each tile come with its stage.
+//                    statistics of each tile come with its stage.  ds and P have
+//                    TMEM columns of their own, so the scores of step t+1 are
+//                    computed as soon as the threads hold those of step t in
+//                    registers, and the gradient MMAs of step t run while they
+//                    work on step t+1.
 //   bwd_dbias_tc     CTA = (128 queries, 64 keys, head); walks every problem row,
 //                    S and dP double-buffered in TMEM, and sums ds in registers:
 //                    the bias gradient is written once per element (no atomics,
@@ -155,17 +155,23 @@ struct RowsArgs {
 // (kDKDV).  A stage per step of 64 columns: the bias tile shared by the rows
 // (128 x 64 bf16, 128-byte swizzle) and per row X1, X2 (64 x 32): K and V
 // (kDQ), Qs and dO (kDKDV), plus for kDKDV the step's -lse2 and -D (64 fp32
-// each).  TMEM per row: S at +0, dP at +64, then ds (bf16, 32 columns) at
-// +128, P (bf16, kDKDV) at +160, and the accumulators: dQ at +160 (kDQ), or
-// dK at +192 and dV at +224 (kDKDV).  ds and P have columns of their own, so
-// the scores of step t+1 are computed while the warps still work on step t.
+// each).
+// kDKDV (kEarly): 2 rows; TMEM per row S at +0, dP at +64, ds (bf16, 32
+// columns) at +128, P (bf16) at +160, dK at +192, dV at +224.  ds and P have
+// columns of their own, so the scores of step t+1 are computed while the warps
+// still work on step t.
+// kDQ: 3 rows; TMEM per row S at +0, dP at +64 (ds as bf16 over its first 32
+// columns, each half written after it was read), dQ at +128; the scores of
+// step t+1 follow the gradient MMA of step t (measured faster for dQ than 2
+// rows with early scores: 1.02 against 1.09 ms per launch at N = 768).
 template <int kMode>
 struct RowsLayout {
-  static constexpr int kR = 2;
-  static constexpr int kRowCols = kMode == kDQ ? 192 : 256;
-  static constexpr int kColDS = 128;
+  static constexpr bool kEarly = kMode == kDKDV;
+  static constexpr int kR = kEarly ? 2 : 3;
+  static constexpr int kRowCols = kEarly ? 256 : 160;
+  static constexpr int kColDS = kEarly ? 128 : 64;
   static constexpr int kColP = 160;
-  static constexpr int kColAcc = kMode == kDQ ? 160 : 192;
+  static constexpr int kColAcc = kEarly ? 192 : 128;
   static constexpr int kStages = 4;
   static constexpr int kProducerWarp = 4 * kR;
   static constexpr int kMmaWarp0 = 4 * kR + 1;  // MMA warp of row g: kMmaWarp0 + g
@@ -359,18 +365,32 @@ __global__ void __launch_bounds__(RowsLayout<kMode>::kThreads, 1)
         issued = true;
       }
       for (int t = 0; ok && t < T; ++t) {
-        if (t + 1 < T) {
-          // S(t+1), dP(t+1) as soon as the warps hold S(t), dP(t) in registers
-          const int s1 = (t + 1) % kStages;
-          if (!(ok = mbar_wait(&st_full[s1], ((t + 1) / kStages) & 1, abort_flag))) break;
-          if (!(ok = mbar_wait(&s_read[g], t & 1, abort_flag))) break;
+        if constexpr (L::kEarly) {
+          if (t + 1 < T) {
+            // S(t+1), dP(t+1) as soon as the warps hold S(t), dP(t) in registers
+            const int s1 = (t + 1) % kStages;
+            if (!(ok = mbar_wait(&st_full[s1], ((t + 1) / kStages) & 1, abort_flag))) break;
+            if (!(ok = mbar_wait(&s_read[g], t & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_sdp(s1);
+          }
+          // the gradient products of step t once ds(t) (and P(t)) are in TMEM
+          if (!(ok = mbar_wait(&ds_full[g], t & 1, abort_flag))) break;
           tc_fence_after();
-          issue_sdp(s1);
+          issue_acc(t % kStages, t == 0);
+        } else {
+          // the gradient product of step t reads ds(t) over dP's columns; S and
+          // dP of step t+1 overwrite them after it (one thread's MMAs run in order)
+          if (!(ok = mbar_wait(&ds_full[g], t & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_acc(t % kStages, t == 0);
+          if (t + 1 < T) {
+            const int s1 = (t + 1) % kStages;
+            if (!(ok = mbar_wait(&st_full[s1], ((t + 1) / kStages) & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_sdp(s1);
+          }
         }
-        // the gradient products of step t once ds(t) (and P(t)) are in TMEM
-        if (!(ok = mbar_wait(&ds_full[g], t & 1, abort_flag))) break;
-        tc_fence_after();
-        issue_acc(t % kStages, t == 0);
       }
       if (ok) mma_commit(&acc_full[g]);
       if (!ok) {
@@ -433,7 +453,7 @@ __global__ void __launch_bounds__(RowsLayout<kMode>::kThreads, 1)
         tmem_ld_wait();
         tmem_regs_ready(sr);
         tmem_regs_ready(dr);
-        if (half == 1) {
+        if (L::kEarly && half == 1) {
           // S(t) and dP(t) are in registers: the MMAs of step t+1 may overwrite them
           tc_fence_before();
           __syncwarp();
@@ -462,7 +482,7 @@ __global__ void __launch_bounds__(RowsLayout<kMode>::kThreads, 1)
           pds[e] = pack_bf16x2(ds.x, ds.y);
           if constexpr (kMode == kDKDV) pp[e] = pack_bf16x2(p.x, p.y);
         }
-        if (half == 0 && t > 0) {
+        if (L::kEarly && half == 0 && t > 0) {
           // ds and P of step t-1 must have been read by its gradient MMAs
           if (!__all_sync(0xffffffffu, mbar_wait(&acc_done[g], (t - 1) & 1, abort_flag))) {
             ok = false;
