@@ -360,6 +360,61 @@ int tri_attn_attention_backward_bf16(const void *Q, const void *K, const void *V
                                      void *workspace, size_t workspace_bytes, void *stream,
                                      unsigned flags);
 
+/* ---- block-level calls (BF16 handle): the 2D grid of devices -------------
+ *
+ * The Design-CP technical summary (§Metodología 1, 2D grid sharding) splits
+ * the pair tensor over a sqrt(P) x sqrt(P) grid of devices and passes K/V
+ * column blocks round a ring with an online softmax.  For a starting-node
+ * block on such a grid, device (a, b) holds the pairs of rows A_a and columns
+ * B_b; its outputs need the K/V of rows A_a over every column block (held
+ * along its grid row) and the logit bias of the pairs (B_b, B_c) for every c.
+ * These calls are the block's three kernels on caller-owned tensors, plus the
+ * merge of partial attention outputs, so that a driver can move K/V, bias and
+ * partial outputs between devices itself.  All device pointers, bf16 unless
+ * stated, 16-byte aligned (lse: 4-byte); asynchronous on `stream`
+ * (TRI_ATTN_FLAG_SYNC waits and returns the device status).  A block of pairs
+ * is Z[rows][cols][c_z], taken as a starting-node problem whose rows are its
+ * rows and whose keys are its columns.  Errors: TRI_ATTN_ERR_INVALID_ARG,
+ * TRI_ATTN_ERR_UNSUPPORTED (F32 handle, rows > 65535, cols > 46340),
+ * TRI_ATTN_ERR_ALIAS (block_gate: out overlaps Z without equalling it),
+ * TRI_ATTN_ERR_NO_DEVICE, TRI_ATTN_ERR_CUDA. */
+
+/* LayerNorm and the projections of every pair of the block: Q, K, V
+ * [rows][H][cols][d] (q scaled by log2(e)/sqrt(d)) and the logit bias
+ * [H][rows][tri_attn_bias_ld(cols)] (times log2(e); -3e38 at keys with
+ * mask[col] == 0 and at columns >= cols).  mask: [cols] or NULL. */
+int tri_attn_block_project(tri_attn_handle *h, const void *Z, int rows, int cols,
+                           const uint8_t *mask, void *Q, void *K, void *V, void *bias,
+                           void *stream, unsigned flags);
+
+/* Flash attention of `rows` problem rows over one key block: o[r][h][j] =
+ * softmax_k(q[r][h][j] . k[r][h][k] + bias[h][j][k]) v[r][h][k] for n queries
+ * and n keys (the tensors of tri_attn_block_project: Q, K, V [rows][H][n][d],
+ * bias [H][n][ld_bias], ld_bias >= tri_attn_bias_ld(n), a multiple of 8, with
+ * its columns n..ld_bias-1 masked), O [rows][H][n][d] normalised within the
+ * block, and lse [rows][H][n] (fp32, natural log of the block's sum; +inf when
+ * the block has no unmasked key) or NULL. */
+int tri_attn_block_attend(tri_attn_handle *h, const void *Q, const void *K, const void *V,
+                          const void *bias, int ld_bias, int rows, int n, void *O, float *lse,
+                          void *stream, unsigned flags);
+
+/* The gate, the output projection and the residual of the block: out =
+ * z + Wo (g * o) + bo with g recomputed from LayerNorm(z); O [rows][H][cols][d],
+ * out [rows][cols][c_z] (out == Z allowed). */
+int tri_attn_block_gate(tri_attn_handle *h, const void *Z, int rows, int cols, const void *O,
+                        void *out, void *stream, unsigned flags);
+
+/* Merge a block's partial output into a running one, for `count` queries:
+ * lse = log(exp(lse_acc) + exp(lse_part)), O_acc = the weighted mean of O_acc
+ * and O_part (weights exp(lse_x - lse)); a part with lse = +inf (no unmasked
+ * key) has weight 0.  With `first` the accumulator is taken as empty (its
+ * contents are not read).  O_acc [count][d] fp32 and lse_acc [count] fp32 are
+ * updated in place; O_part [count][d] bf16, lse_part [count] fp32; O_out
+ * [count][d] bf16 receives the merged output, or NULL.  No handle. */
+int tri_attn_merge_partial(float *O_acc, float *lse_acc, const void *O_part,
+                           const float *lse_part, long long count, int first, void *O_out,
+                           void *stream, unsigned flags);
+
 /* Release everything the handle owns.  NULL-safe.  Not stream-ordered:
  * call it after the work that uses the handle has completed. */
 int tri_attn_destroy(tri_attn_handle *h);

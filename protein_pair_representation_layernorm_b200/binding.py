@@ -96,6 +96,10 @@ def lib() -> ctypes.CDLL:
         L.tri_attn_bias_ld.argtypes = [ci]
         L.tri_attn_rows_bias.argtypes = [vp, vp, ci, ci, ci, vp, vp, vp, cu]
         L.tri_attn_rows_forward.argtypes = [vp, vp, ci, ci, ci, vp, vp, vp, vp, cu]
+        L.tri_attn_block_project.argtypes = [vp, vp, ci, ci, vp, vp, vp, vp, vp, vp, cu]
+        L.tri_attn_block_attend.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, vp, vp, vp, cu]
+        L.tri_attn_block_gate.argtypes = [vp, vp, ci, ci, vp, vp, vp, cu]
+        L.tri_attn_merge_partial.argtypes = [vp, vp, vp, vp, ctypes.c_longlong, ci, vp, vp, cu]
         L.tri_attn_attention_backward_workspace_bytes.argtypes = [ci, ci]
         L.tri_attn_attention_backward_workspace_bytes.restype = sz
         L.tri_attn_attention_backward.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, vp, vp, vp, vp,
@@ -374,6 +378,51 @@ class TriangleAttention:
             raise TriAttnError(rc, "tri_attn_rows_forward")
         return out
 
+    # ------------------------------------------------ block-level calls (bf16)
+    def block_project(self, Z_blk: torch.Tensor, mask=None, stream=None, flags: int = 0):
+        """(Q, K, V, bias, ld) of a block of pairs Z_blk [rows][cols][c_z]:
+        Q, K, V [rows][H][cols][d] (q scaled by log2(e)/sqrt(d)), bias
+        [H][rows][ld] (times log2(e), -3e38 at masked keys and padding)."""
+        assert Z_blk.is_cuda and Z_blk.dtype == torch.bfloat16 and Z_blk.is_contiguous()
+        rows, cols = Z_blk.shape[0], Z_blk.shape[1]
+        ld = self.bias_ld(cols)
+        Q, K, V = (torch.empty(rows, 4, cols, 32, dtype=torch.bfloat16, device=Z_blk.device)
+                   for _ in range(3))
+        bias = torch.empty(4, rows, ld, dtype=torch.bfloat16, device=Z_blk.device)
+        if mask is not None:
+            mask = mask.to(device=Z_blk.device, dtype=torch.uint8).contiguous()
+        rc = lib().tri_attn_block_project(self.handle, _ptr(Z_blk), rows, cols, _ptr(mask),
+                                          _ptr(Q), _ptr(K), _ptr(V), _ptr(bias),
+                                          _stream_handle(stream), flags)
+        if rc != TRI_ATTN_OK:
+            raise TriAttnError(rc, "tri_attn_block_project")
+        return Q, K, V, bias, ld
+
+    def block_attend(self, Q, K, V, bias, ld: int, stream=None, flags: int = 0):
+        """(O, lse) of the rows' queries over one key block (O bf16
+        [rows][H][n][d] normalised within the block, lse fp32 [rows][H][n])."""
+        rows, _, n, _ = Q.shape
+        O = torch.empty_like(Q)
+        lse = torch.empty(rows, 4, n, dtype=torch.float32, device=Q.device)
+        rc = lib().tri_attn_block_attend(self.handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(bias),
+                                         int(ld), rows, n, _ptr(O), _ptr(lse),
+                                         _stream_handle(stream), flags)
+        if rc != TRI_ATTN_OK:
+            raise TriAttnError(rc, "tri_attn_block_attend")
+        return O, lse
+
+    def block_gate(self, Z_blk: torch.Tensor, O: torch.Tensor, out=None, stream=None,
+                   flags: int = 0):
+        """out = z + Wo (g * o) + bo for the block's pairs."""
+        rows, cols = Z_blk.shape[0], Z_blk.shape[1]
+        if out is None:
+            out = torch.empty_like(Z_blk)
+        rc = lib().tri_attn_block_gate(self.handle, _ptr(Z_blk), rows, cols, _ptr(O), _ptr(out),
+                                       _stream_handle(stream), flags)
+        if rc != TRI_ATTN_OK:
+            raise TriAttnError(rc, "tri_attn_block_gate")
+        return out
+
     def status(self, stream=None) -> int:
         return tri_attn_get_status(self.handle, _stream_handle(stream))
 
@@ -452,6 +501,19 @@ def attention_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, bias: t
     if rc != TRI_ATTN_OK:
         raise TriAttnError(rc, "tri_attn_attention_forward")
     return O, lse
+
+
+def merge_partial(O_acc: torch.Tensor, lse_acc: torch.Tensor, O_part: torch.Tensor,
+                  lse_part: torch.Tensor, first: bool, O_out: torch.Tensor | None = None,
+                  stream=None):
+    """Merge one key block's (O_part bf16, lse_part) into the running (O_acc
+    fp32, lse_acc), in place; O_out (bf16) receives the merged output."""
+    count = lse_part.numel()
+    rc = lib().tri_attn_merge_partial(_ptr(O_acc), _ptr(lse_acc), _ptr(O_part), _ptr(lse_part),
+                                      count, 1 if first else 0, _ptr(O_out),
+                                      _stream_handle(stream), 0)
+    if rc != TRI_ATTN_OK:
+        raise TriAttnError(rc, "tri_attn_merge_partial")
 
 
 def _core_checked_bf16(Q, K, V, bias, *more):

@@ -32,6 +32,7 @@
 #include "common.cuh"
 #include "gate_out.cuh"
 #include "kernels_f32.cuh"
+#include "merge.cuh"
 #include "pair_ln_proj.cuh"
 #include "sm100.cuh"
 #include "tri_attn_fwd.cuh"
@@ -1579,4 +1580,188 @@ extern "C" int tri_attn_attention_backward_bf16(const void* Q, const void* K, co
     CUDA_TRY(cudaGetLastError());
   }
   return core_finish(w, st, flags);
+}
+
+// ------------------------------------------------------------------ block-level calls
+// The three kernels of the block on caller-owned tensors, for a distributed
+// driver that moves the intermediate tensors between devices itself (the 2D
+// grid: K/V column blocks passed round a ring, partial outputs merged by
+// their log-sum-exp).  A block of pairs is [rows][cols][c_z], taken as a
+// starting-node problem whose rows are its rows and whose keys are its columns.
+namespace {
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int check_block_handle(tri_attn_handle* h, int rows, int cols) {
+  if (!h || rows < 1 || cols < 1) return TRI_ATTN_ERR_INVALID_ARG;
+  if (h->dtype != TRI_ATTN_BF16) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (rows > 65535 || cols > 46340) return TRI_ATTN_ERR_UNSUPPORTED;
+  return TRI_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int tri_attn_block_project(tri_attn_handle* h, const void* Z, int rows, int cols,
+                                      const uint8_t* mask, void* Q, void* K, void* V, void* bias,
+                                      void* stream, unsigned flags) {
+  int rc = check_block_handle(h, rows, cols);
+  if (rc != TRI_ATTN_OK) return rc;
+  if (!aligned16(Z) || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(bias))
+    return TRI_ATTN_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+  rc = set_kernel_attrs();
+  if (rc != TRI_ATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  tri::ProjArgs a{};
+  a.Z = static_cast<const bf16*>(Z);
+  a.mask = mask;
+  a.N = cols;
+  a.orient = 0;
+  a.row0 = 0;
+  a.rows = rows;
+  a.write_qkv = 1;
+  a.write_bias = 1;
+  a.w_img = static_cast<const uint8_t*>(h->w_qkvg);
+  a.w_b = h->w_b;
+  a.gamma = h->gamma;
+  a.beta = h->beta;
+  a.eps = h->eps;
+  a.q_scale = h->q_scale;
+  a.Q = static_cast<bf16*>(Q);
+  a.K = static_cast<bf16*>(K);
+  a.V = static_cast<bf16*>(V);
+  a.bias = static_cast<bf16*>(bias);
+  a.ld_bias = ld_bias_for(cols);
+  a.z_row0 = 0;
+  a.bias_row0 = 0;
+  a.bias_rows = rows;
+  a.debug_stall = (flags & TRI_ATTN_FLAG_DEBUG_STALL_PROJ) ? 1 : 0;
+  a.status = h->status;
+  const long long ntiles = static_cast<long long>(rows) * ((cols + 127) / 128);
+  const unsigned grid = static_cast<unsigned>(std::min<long long>(
+      (ntiles + tri::plp::kGroupsPerCta - 1) / tri::plp::kGroupsPerCta, h->num_sms));
+  CUtensorMap mz;
+  if (!make_map_3d(&mz, Z, kCz, cols, rows, kCz * 2, static_cast<uint64_t>(cols) * kCz * 2, 64,
+                   128, CU_TENSOR_MAP_SWIZZLE_128B, 1))
+    return TRI_ATTN_ERR_CUDA;
+  tri::plp::pair_ln_proj<<<grid, tri::plp::kThreads, tri::plp::kSmemBytes, st>>>(mz, a);
+  CUDA_TRY(cudaGetLastError());
+  return finish_call(h, st, flags);
+}
+
+extern "C" int tri_attn_block_attend(tri_attn_handle* h, const void* Q, const void* K,
+                                     const void* V, const void* bias, int ld_bias, int rows,
+                                     int n, void* O, float* lse, void* stream, unsigned flags) {
+  int rc = check_block_handle(h, rows, n);
+  if (rc != TRI_ATTN_OK) return rc;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(bias) || !aligned16(O) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3)) || ld_bias < ld_bias_for(n) ||
+      ld_bias % 8 != 0)
+    return TRI_ATTN_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+  rc = set_kernel_attrs();
+  if (rc != TRI_ATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CUtensorMap mq, mk, mv, mb;
+  const uint64_t rh = static_cast<uint64_t>(rows) * kHeads;
+  const uint64_t row_stride = static_cast<uint64_t>(n) * kD * 2;
+  if (!make_map_3d(&mq, Q, kD, n, rh, kD * 2, row_stride, kD, tri::attn::kBJ,
+                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_3d(&mk, K, kD, n, rh, kD * 2, row_stride, kD, tri::attn::kBK,
+                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_3d(&mv, V, kD, n, rh, kD * 2, row_stride, kD, tri::attn::kBK,
+                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_3d(&mb, bias, ld_bias, n, kHeads, static_cast<uint64_t>(ld_bias) * 2,
+                   static_cast<uint64_t>(n) * ld_bias * 2, tri::attn::kBK, tri::attn::kBJ,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return TRI_ATTN_ERR_CUDA;
+  tri::AttnArgs a{};
+  a.O = static_cast<bf16*>(O);
+  a.lse = lse;
+  a.N = n;
+  a.rows = rows;
+  a.debug_stall = (flags & TRI_ATTN_FLAG_DEBUG_STALL) ? 1 : 0;
+  a.status = h->status;
+  const dim3 grid((n + tri::attn::kBJ - 1) / tri::attn::kBJ,
+                  (rows + tri::attn::kRows - 1) / tri::attn::kRows, kHeads);
+  tri::attn::tri_attn_fwd<<<grid, tri::attn::kThreads, tri::attn::kSmemBytes, st>>>(mq, mk, mv,
+                                                                                 mb, a);
+  CUDA_TRY(cudaGetLastError());
+  return finish_call(h, st, flags);
+}
+
+extern "C" int tri_attn_block_gate(tri_attn_handle* h, const void* Z, int rows, int cols,
+                                   const void* O, void* out, void* stream, unsigned flags) {
+  int rc = check_block_handle(h, rows, cols);
+  if (rc != TRI_ATTN_OK) return rc;
+  if (!aligned16(Z) || !aligned16(O) || !aligned16(out)) return TRI_ATTN_ERR_INVALID_ARG;
+  {
+    // out may be Z itself; any other overlap is rejected
+    const size_t bytes = static_cast<size_t>(rows) * cols * kCz * 2;
+    const char* z0 = static_cast<const char*>(Z);
+    const char* o0 = static_cast<const char*>(out);
+    if (o0 != z0 && o0 < z0 + bytes && z0 < o0 + bytes) return TRI_ATTN_ERR_ALIAS;
+  }
+  if (cudaSetDevice(h->device) != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+  rc = set_kernel_attrs();
+  if (rc != TRI_ATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CUtensorMap mo, mz, mout;
+  const uint64_t rowb = static_cast<uint64_t>(cols) * kCz * 2;
+  if (!make_map_3d(&mo, O, kD, cols, static_cast<uint64_t>(rows) * kHeads, kD * 2,
+                   static_cast<uint64_t>(cols) * kD * 2, kD, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_3d(&mz, Z, kCz, cols, rows, kCz * 2, rowb, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B,
+                   1) ||
+      !make_map_3d(&mout, out, kCz, cols, rows, kCz * 2, rowb, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B, 1))
+    return TRI_ATTN_ERR_CUDA;
+  tri::GateArgs a{};
+  a.Z = static_cast<const bf16*>(Z);
+  a.O = static_cast<const bf16*>(O);
+  a.wo_img = static_cast<const uint8_t*>(h->w_o);
+  a.wg_img = static_cast<const uint8_t*>(h->w_g);
+  a.b_o = h->b_o;
+  a.b_g = h->b_g;
+  a.gamma = h->gamma;
+  a.beta = h->beta;
+  a.eps = h->eps;
+  a.out = static_cast<bf16*>(out);
+  a.N = cols;
+  a.orient = 0;
+  a.row0 = 0;
+  a.rows = rows;
+  a.z_row0 = 0;
+  a.debug_stall = (flags & TRI_ATTN_FLAG_DEBUG_STALL_GATE) ? 1 : 0;
+  a.status = h->status;
+  const long long ntiles = static_cast<long long>(rows) * ((cols + 127) / 128);
+  const unsigned grid = static_cast<unsigned>(std::min<long long>(ntiles, h->num_sms));
+  tri::gout::gate_out<<<grid, tri::gout::kThreads, tri::gout::kSmemBytes, st>>>(mo, mz, mout, a);
+  CUDA_TRY(cudaGetLastError());
+  return finish_call(h, st, flags);
+}
+
+extern "C" int tri_attn_merge_partial(float* O_acc, float* lse_acc, const void* O_part,
+                                      const float* lse_part, long long count, int first,
+                                      void* O_out, void* stream, unsigned flags) {
+  if (!aligned16(O_acc) || !aligned16(O_part) || !lse_acc || !lse_part || count < 1 ||
+      (O_out && !aligned16(O_out)) || (reinterpret_cast<uintptr_t>(lse_acc) & 3) ||
+      (reinterpret_cast<uintptr_t>(lse_part) & 3))
+    return TRI_ATTN_ERR_INVALID_ARG;
+  int rc = check_device();
+  if (rc != TRI_ATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  tri::merge::MergeArgs a{};
+  a.o_acc = O_acc;
+  a.lse_acc = lse_acc;
+  a.o_part = static_cast<const bf16*>(O_part);
+  a.lse_part = lse_part;
+  a.o_out = static_cast<bf16*>(O_out);
+  a.count = count;
+  a.first = first ? 1 : 0;
+  const long long blocks = (count + tri::merge::kThreads - 1) / tri::merge::kThreads;
+  if (blocks > 0x7fffffffLL) return TRI_ATTN_ERR_UNSUPPORTED;
+  tri::merge::merge_partial<<<static_cast<unsigned>(blocks), tri::merge::kThreads, 0, st>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  if (flags & TRI_ATTN_FLAG_SYNC) CUDA_TRY(cudaStreamSynchronize(st));
+  return TRI_ATTN_OK;
 }

@@ -208,3 +208,21 @@ def test_tensor_core_core_calls_reject_bad_arguments_without_device():
         assert f() == binding.TRI_ATTN_ERR_NO_DEVICE
         assert f(lse=None) == binding.TRI_ATTN_ERR_NO_DEVICE  # lse is optional in the forward
         assert b() == binding.TRI_ATTN_ERR_NO_DEVICE
+
+
+def test_block_calls_reject_bad_arguments_without_device():
+    L = binding.lib()
+    buf, bad = 0x10000, binding.TRI_ATTN_ERR_INVALID_ARG
+    # no handle
+    assert L.tri_attn_block_project(None, buf, 8, 8, None, buf, buf, buf, buf, None, 0) == bad
+    assert L.tri_attn_block_attend(None, buf, buf, buf, buf, 64, 8, 8, buf, buf, None, 0) == bad
+    assert L.tri_attn_block_gate(None, buf, 8, 8, buf, buf, None, 0) == bad
+    # the merge needs no handle: pointers, alignment and count are checked first
+    assert L.tri_attn_merge_partial(None, buf, buf, buf, 10, 1, None, None, 0) == bad
+    assert L.tri_attn_merge_partial(buf + 4, buf, buf, buf, 10, 1, None, None, 0) == bad
+    assert L.tri_attn_merge_partial(buf, buf, buf, buf, 0, 1, None, None, 0) == bad
+    assert L.tri_attn_merge_partial(buf, buf + 2, buf, buf, 10, 1, None, None, 0) == bad
+    assert L.tri_attn_merge_partial(buf, buf, buf, buf, 10, 1, buf + 8, None, 0) == bad
+    if not torch.cuda.is_available():
+        assert L.tri_attn_merge_partial(buf, buf, buf, buf, 10, 1, None, None, 0) == \
+            binding.TRI_ATTN_ERR_NO_DEVICE
