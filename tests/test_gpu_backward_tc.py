@@ -54,8 +54,8 @@ def _gpu(q, k, v, g, bias, mask):
     O, lse = binding.attention_forward_bf16(Q, K, V, B, m)
     grads = binding.attention_backward_bf16(Q, K, V, B, O, lse, G, m, sync=True)
     torch.cuda.synchronize()
-    return O.float().cpu().numpy(), lse.cpu().numpy(), [t.cpu().numpy().astype(np.float64)
-                                                        for t in grads]
+    # fp32 as computed (the comparisons promote to fp64)
+    return O.float().cpu().numpy(), lse.cpu().numpy(), [t.cpu().numpy() for t in grads]
 
 
 def _f64(t):
@@ -131,26 +131,32 @@ def test_tensor_core_backward_is_deterministic():
         assert np.array_equal(x, y)
 
 
-def test_tensor_core_full_size_sampled():
-    """N = 768 with every row: rows 0, 383 and 767 of dQ, dK, dV and query
-    lines 0, 400 and 767 of the bias gradient (summed over all 768 rows)
-    against the oracle; sum_k dbias[h][j][k] = 0 for every (h, j)."""
-    N, rows = 768, 768
+@pytest.mark.parametrize("N", [768, 1536])
+def test_tensor_core_full_size_sampled(N):
+    """Every row at N = 768 and at N = 1536 (the size bench.py --backward
+    times): rows 0, N/2 - 1 and N - 1 of dQ, dK, dV and query lines 0, N/2 + 16
+    and N - 1 of the bias gradient (summed over all N rows) against the
+    oracle; sum_k dbias[h][j][k] = 0 for every (h, j)."""
+    rows = N
     q, k, v, g, bias, mask = _inputs(19, rows, N, "random")
     _, _, (dq, dk, dv, db) = _gpu(q, k, v, g, bias, mask)
-    qo, ko, vo, go = (_to_oracle(_f64(t)) for t in (q, k, v, g))
+    row = lambda t, r: t[r].float().numpy().transpose(1, 0, 2).astype(np.float64)  # noqa: E731
     b = _f64(bias)
-    for r in (0, 383, 767):
-        rq, rk, rv, _ = oracle.attend_bwd(qo[r], ko[r], vo[r], b, go[r], mask)
-        _check(f"dQ N=768 row {r}", _to_oracle(dq)[r], rq)
-        _check(f"dK N=768 row {r}", _to_oracle(dk)[r], rk)
-        _check(f"dV N=768 row {r}", _to_oracle(dv)[r], rv)
-    for j in (0, 400, 767):
-        ref = np.zeros((H, N))
-        for r in range(rows):
-            ref += oracle.attend_bwd(qo[r][j:j + 1], ko[r], vo[r], b[:, j:j + 1, :],
-                                     go[r][j:j + 1], mask)[3][:, 0, :]
-        _check(f"dbias N=768 line {j}", db[:, j, :], ref)
+    for r in (0, N // 2 - 1, N - 1):
+        rq, rk, rv, _ = oracle.attend_bwd(row(q, r), row(k, r), row(v, r), b, row(g, r), mask)
+        _check(f"dQ N={N} row {r}", dq[r].transpose(1, 0, 2), rq)
+        _check(f"dK N={N} row {r}", dk[r].transpose(1, 0, 2), rk)
+        _check(f"dV N={N} row {r}", dv[r].transpose(1, 0, 2), rv)
+    lines = (0, N // 2 + 16, N - 1)
+    refs = {j: np.zeros((H, N)) for j in lines}
+    for r in range(rows):
+        kr, vr = row(k, r), row(v, r)
+        qr, gr = row(q, r), row(g, r)
+        for j in lines:
+            refs[j] += oracle.attend_bwd(qr[j:j + 1], kr, vr, b[:, j:j + 1, :], gr[j:j + 1],
+                                         mask)[3][:, 0, :]
+    for j in lines:
+        _check(f"dbias N={N} line {j}", db[:, j, :], refs[j])
     row_sums = np.abs(db.sum(axis=2)).max()
     assert row_sums <= 1e-3 * np.abs(db).sum(axis=2).max(), row_sums
 
