@@ -84,3 +84,50 @@ def test_merge_of_split_keys_equals_one_block():
     rel = ((out.float() - O_all.float()).norm() / O_all.float().norm()).item()
     assert rel < 5e-3, rel
     blk.close()
+
+
+@pytest.mark.parametrize("masked", ["first_block", "all"])
+def test_grid_with_fully_masked_key_blocks(masked):
+    """A key block whose every key is masked has lse = +inf and weight 0 in the
+    merge; with every key masked o = 0 and out = z + bo (bo = 0 here)."""
+    N, p = 256, 2
+    inp = workloads.make_inputs(N, "bf16", 150, "random:0.1")
+    mask = torch.ones(N, dtype=torch.uint8)
+    if masked == "first_block":
+        mask[: N // p] = 0
+    else:
+        mask[:] = 0
+    inp = workloads.Inputs(**{**{f: getattr(inp, f) for f in (
+        "Z", "gamma", "beta", "Wq", "Wk", "Wv", "Wg", "bg", "Wb", "Wo", "bo")}, "mask": mask})
+    blk = binding.TriangleAttention(inp.weights(), dtype=torch.bfloat16)
+    for orientation in (0, 1):
+        got = _grid(inp, blk, p, orientation)
+        if masked == "all":
+            assert torch.equal(got.contiguous().view(torch.int16), inp.Z.cuda().view(torch.int16))
+        else:
+            ref = oracle.tri_attn_full(to_problem(inp), orientation)
+            st = compare(got.double().cpu().numpy(), ref, inp.Z.double().numpy(), "bf16")
+            assert_within(st, "bf16", f"2D grid, first key block masked, orientation {orientation}")
+    blk.close()
+
+
+def test_block_gate_in_place():
+    N = 128
+    inp = workloads.make_inputs(N, "bf16", 160, "random:0.1")
+    blk = binding.TriangleAttention(inp.weights(), dtype=torch.bfloat16)
+    Z = inp.Z.cuda()
+    Q, K, V, bias, ld = blk.block_project(Z, inp.mask.cuda())
+    O, _ = blk.block_attend(Q, K, V, bias, ld)
+    want = blk.block_gate(Z, O)
+    Z2 = Z.clone()
+    got = blk.block_gate(Z2, O, out=Z2)
+    torch.cuda.synchronize()
+    assert got.data_ptr() == Z2.data_ptr()
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+    # an output that overlaps Z without being Z (one row of pairs apart) is rejected
+    big = torch.empty(N + 1, N, 128, dtype=torch.bfloat16, device="cuda")
+    big[:N].copy_(Z)
+    with pytest.raises(binding.TriAttnError) as err:
+        blk.block_gate(big[:N], O, out=big[1:])
+    assert err.value.code == binding.TRI_ATTN_ERR_ALIAS
+    blk.close()
