@@ -101,6 +101,16 @@ def test_workload1_full(orientation):
 
 
 @pytest.mark.parametrize("orientation", [0, 1])
+@pytest.mark.parametrize("w", [2, 3])
+def test_workload_full_tensor(w, orientation):
+    """Every line of the block's output (and of the attention output o) at
+    N = 768 (three chains) and N = 1536 (the benchmark's size) against the
+    oracle: a few minutes of fp64 on the host's cores."""
+    inp = _workload(w)
+    _check_full(inp, orientation, "bf16", f"workload {w} (N={inp.N}) full {NAMES[orientation]}")
+
+
+@pytest.mark.parametrize("orientation", [0, 1])
 @pytest.mark.parametrize("w", [2, 3, 4])
 def test_workload_sampled(w, orientation):
     inp = _workload(w)
