@@ -304,6 +304,18 @@ def run_ours(args, world, rank, local):
     kms, kn = blk.kernel_times()
     rc = blk.status(st)
     assert rc == binding.TRI_ATTN_OK, binding.tri_attn_status_string(rc)
+    # each orientation's kernels on their own, outside the timed region: 20
+    # blocks of one orientation at a time, per-kernel CUDA events
+    by_orient = {}
+    for name, orient, src, dst in (("starting", binding.TRI_ATTN_STARTING, Z, out1),
+                                   ("ending", binding.TRI_ATTN_ENDING, out1, out2)):
+        with torch.cuda.stream(st):
+            for _ in range(20):
+                blk.forward(src, orient, mask, out=dst, stream=st, flags=TIME)
+        st.synchronize()
+        oms, on = blk.kernel_times()
+        by_orient[name] = {k: oms[i] / max(on[i], 1)
+                           for i, k in enumerate(("pair_ln_proj", "tri_attn_fwd", "gate_out"))}
 
     value = world * flops_step * args.steps / (t_ms_max / 1e3) / 1e12
     peak_tf, peak_gbs, peak_src = measured_peaks()
@@ -395,6 +407,7 @@ def run_ours(args, world, rank, local):
             "gate_out": {"ms": gate_ms, "launches": kn[2],
                          "GB/s": gate_bytes / (gate_ms / 1e3) / 1e9,
                          "frac_hbm": gate_bytes / (gate_ms / 1e3) / 1e9 / peak_gbs},
+            "ms_by_orientation": by_orient,
         },
         "pair_rows_per_s": world * 2 * N * args.steps / (t_ms_max / 1e3),
         "clocks": clk,
