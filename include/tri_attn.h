@@ -55,8 +55,7 @@ extern "C" {
 #define TRI_ATTN_ERR_UNSUPPORTED   -2  /* shape or dtype the kernels do not cover */
 #define TRI_ATTN_ERR_ALIAS         -3  /* out overlaps Z without being equal to it */
 #define TRI_ATTN_ERR_OOM           -4  /* device or host allocation failed */
-#define TRI_ATTN_ERR_CUDA          -5  /* a CUDA runtime call or launch failed (also as device
-                                         status: a kernel found its launch unusable) */
+#define TRI_ATTN_ERR_CUDA          -5  /* a CUDA runtime call or launch failed */
 #define TRI_ATTN_ERR_TIMEOUT       -6  /* a kernel's bounded wait expired (device status) */
 #define TRI_ATTN_ERR_NO_DEVICE     -7  /* no sm_100 device is available */
 

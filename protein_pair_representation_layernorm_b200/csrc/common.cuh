@@ -94,7 +94,6 @@ struct GateArgs {
 };
 
 // Device status word values (mirror the public codes).
-constexpr int kStatusBadLaunch = -5;  // TRI_ATTN_ERR_CUDA: a kernel found its launch unusable
 constexpr int kStatusTimeout = -6;
 
 __device__ __forceinline__ void report_status(int* status, int code) {
